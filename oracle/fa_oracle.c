@@ -1,0 +1,155 @@
+/*
+ * fa_oracle.c -- fp64 reference for the exact attention forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or
+ * calls this file: only the tests, the package smoke check and the CPU
+ * baseline leg of the benchmark do.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes is the plain definition of attention that the pages
+ * state as "standard attention" (Chapter 15 -- FlashAttention, section
+ * "Standard vs Flash Attention", left column, steps 1-4):
+ *
+ *     S = scale * Q K^T          full rows of the score matrix, in fp64
+ *     causal: s_ij = -inf for j > i
+ *     P = softmax(S)             two passes over each row: max, then exp/sum
+ *     O = P V
+ *     lse_i = m_i + ln(sum_j exp(s_ij - m_i))     natural log
+ *
+ * The pages never write the scale, the causal mask or the log-sum-exp
+ * output; those come from the workload definition and are applied in the
+ * plainest way (scale multiplies Q K^T before softmax; the causal mask keeps
+ * keys j <= i; lse is the natural log of the row's softmax denominator in
+ * scaled units).  Exactness is what the method promises (Chapter 15 --
+ * FlashAttention, "Key Takeaways: Online Softmax Enables It": exact results,
+ * no approximation), so the oracle is the definition, not the tiled
+ * algorithm.
+ *
+ * Memory: the score rows of one head are materialised in blocks of at most
+ * ORACLE_ROW_BLOCK rows by N columns.  That bounds memory only; every row is
+ * still the full, two-pass, non-online computation.
+ *
+ * Inputs are fp32 arrays holding the exact values the GPU reads (bf16 values
+ * are exactly representable in fp32); every arithmetic step is in fp64.
+ * Layout: q, k, v are contiguous [BH][N][d]; o is [BH][nrows][d] fp64 and
+ * lse is [BH][nrows] fp64, one entry per requested row.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_ROW_BLOCK 64
+
+int oracle_version(void) { return 1; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * One block of rows of one head.
+ *   q_rows: the requested query rows (indices into [0, n)), count nr <= ORACLE_ROW_BLOCK
+ *   s:      scratch of nr * n doubles (the materialised score rows)
+ */
+static void attention_row_block(const float* q, const float* k, const float* v,
+                                int64_t n, int64_t d, double scale, int causal,
+                                const int64_t* q_rows, int64_t nr, double* s,
+                                double* o_out, double* lse_out) {
+    /* Step 1: S = scale * Q K^T for the requested rows, masked. */
+    for (int64_t r = 0; r < nr; ++r) {
+        const int64_t i = q_rows[r];
+        const float* qi = q + i * d;
+        double* srow = s + r * n;
+        for (int64_t j = 0; j < n; ++j) {
+            if (causal && j > i) {
+                srow[j] = -INFINITY;
+                continue;
+            }
+            const float* kj = k + j * d;
+            double dot = 0.0;
+            for (int64_t t = 0; t < d; ++t) dot += (double)qi[t] * (double)kj[t];
+            srow[j] = scale * dot;
+        }
+    }
+    /* Steps 2-3: P = softmax(S), first pass the row max, second pass the sum. */
+    for (int64_t r = 0; r < nr; ++r) {
+        double* srow = s + r * n;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j)
+            if (srow[j] > m) m = srow[j];
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            srow[j] = exp(srow[j] - m); /* exp(-inf) = 0 for masked keys */
+            l += srow[j];
+        }
+        for (int64_t j = 0; j < n; ++j) srow[j] /= l; /* srow now holds P */
+        lse_out[r] = m + log(l);
+    }
+    /* Step 4: O = P V, summed over the keys the mask allows. */
+    for (int64_t r = 0; r < nr; ++r) {
+        const double* prow = s + r * n;
+        double* orow = o_out + r * d;
+        const int64_t j_end = causal ? q_rows[r] + 1 : n;
+        for (int64_t t = 0; t < d; ++t) orow[t] = 0.0;
+        for (int64_t j = 0; j < j_end; ++j) {
+            const double p = prow[j];
+            const float* vj = v + j * d;
+            for (int64_t t = 0; t < d; ++t) orow[t] += p * (double)vj[t];
+        }
+    }
+}
+
+/*
+ * oracle_attention_fwd
+ *   q, k, v:  [bh][n][d] fp32 (exact input values)
+ *   rows:     [bh][nrows] int64 row indices per head (each in [0, n))
+ *   o:        [bh][nrows][d] fp64 output
+ *   lse:      [bh][nrows] fp64 output (natural log)
+ * Returns 0 on success, -1 on bad arguments, -2 if scratch cannot be allocated.
+ */
+int oracle_attention_fwd(const float* q, const float* k, const float* v,
+                         int64_t bh, int64_t n, int64_t d, double scale, int causal,
+                         const int64_t* rows, int64_t nrows, double* o, double* lse) {
+    if (!q || !k || !v || !rows || !o || !lse) return -1;
+    if (bh <= 0 || n <= 0 || d <= 0 || nrows <= 0) return -1;
+    for (int64_t x = 0; x < bh * nrows; ++x)
+        if (rows[x] < 0 || rows[x] >= n) return -1;
+
+    const int64_t nblocks = (nrows + ORACLE_ROW_BLOCK - 1) / ORACLE_ROW_BLOCK;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* s = NULL;
+        int64_t s_rows = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t task = 0; task < bh * nblocks; ++task) {
+            const int64_t h = task / nblocks;
+            const int64_t b0 = (task % nblocks) * ORACLE_ROW_BLOCK;
+            const int64_t nr = (nrows - b0 < ORACLE_ROW_BLOCK) ? nrows - b0 : ORACLE_ROW_BLOCK;
+            if (s_rows < nr) {
+                free(s);
+                s = (double*)malloc((size_t)(nr * n) * sizeof(double));
+                s_rows = s ? nr : 0;
+            }
+            if (!s) {
+#pragma omp atomic write
+                failed = 1;
+                continue;
+            }
+            const int64_t head = h * n * d;
+            attention_row_block(q + head, k + head, v + head, n, d, scale, causal,
+                                rows + h * nrows + b0, nr, s,
+                                o + (h * nrows + b0) * d, lse + h * nrows + b0);
+        }
+        free(s);
+    }
+    return failed ? -2 : 0;
+}

@@ -1,0 +1,273 @@
+"""Pins for the fp64 oracle: checks against facts fixed outside the oracle.
+
+Each ``pin_*`` function takes a loaded oracle library (the real one, or a
+deliberately broken copy built by the mutation tests) and raises
+AssertionError when the oracle disagrees with the fact it pins.  None of them
+restates the oracle's own formula: they use closed forms, invariances of the
+definition, the online-softmax ledger the pages describe (FlashAttention,
+Playable, EP 04), hand-worked tiny cases and torch's own fp64 attention.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+
+RNG_SEED = 1234
+
+
+def _rand(shape, seed, scale=1.0):
+    g = np.random.default_rng(seed)
+    return (g.standard_normal(shape) * scale).astype(np.float32)
+
+
+def _run(lib, q, k, v, scale, causal, rows=None):
+    return oracle.attention_fwd(q, k, v, scale, causal, rows=rows, lib=lib)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def pin_hand_worked(lib):
+    """N=2, d=1, scale=1, worked by hand.
+
+    q = [ln 3, 0], k = [1, 0], v = [4, 8]:
+      row 0 scores [ln 3, 0] -> softmax [3/4, 1/4] -> o = 3 + 2 = 5, lse = ln 4
+      row 1 scores [0, 0]    -> softmax [1/2, 1/2] -> o = 6,         lse = ln 2
+    causal: row 0 sees only key 0 -> o = 4, lse = ln 3; row 1 unchanged.
+    """
+    q = np.array([math.log(3.0), 0.0], dtype=np.float64)
+    # ln 3 is not exact in fp32; carry the fp32 value through the hand result.
+    q32 = q.astype(np.float32)
+    a = float(q32[0])  # the score of row 0 against key 0
+    Q = q32.reshape(1, 1, 2, 1)
+    K = np.array([1.0, 0.0], dtype=np.float32).reshape(1, 1, 2, 1)
+    V = np.array([4.0, 8.0], dtype=np.float32).reshape(1, 1, 2, 1)
+    o, lse = _run(lib, Q, K, V, 1.0, False)
+    w0 = math.exp(a) / (math.exp(a) + 1.0)
+    assert abs(o[0, 0, 0, 0] - (4 * w0 + 8 * (1 - w0))) < 1e-13, o
+    assert abs(o[0, 0, 0, 0] - 5.0) < 1e-6
+    assert abs(o[0, 0, 1, 0] - 6.0) < 1e-14
+    assert abs(lse[0, 0, 0] - math.log(math.exp(a) + 1.0)) < 1e-14
+    assert abs(lse[0, 0, 1] - math.log(2.0)) < 1e-14
+    o, lse = _run(lib, Q, K, V, 1.0, True)
+    assert o[0, 0, 0, 0] == 4.0
+    assert abs(lse[0, 0, 0] - a) < 1e-14
+    assert abs(o[0, 0, 1, 0] - 6.0) < 1e-14
+    assert abs(lse[0, 0, 1] - math.log(2.0)) < 1e-14
+
+
+def pin_q_zero_mean_of_v(lib):
+    """Q = 0 makes every score equal: O_i is the mean of the allowed V rows and
+    lse_i = ln(#allowed keys), whatever the scale."""
+    B, H, N, d = 1, 2, 37, 8
+    q = np.zeros((B, H, N, d), np.float32)
+    k = _rand((B, H, N, d), 1)
+    v = _rand((B, H, N, d), 2)
+    for causal in (False, True):
+        o, lse = _run(lib, q, k, v, 0.7, causal)
+        for i in range(N):
+            n_allowed = i + 1 if causal else N
+            want = v[:, :, :n_allowed].astype(np.float64).mean(axis=2)
+            np.testing.assert_allclose(o[:, :, i], want, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lse[:, :, i], math.log(n_allowed), rtol=0, atol=1e-13)
+
+
+def pin_single_key(lib):
+    """N = 1: the only key gets weight 1, so O = V_0 and lse = scale * q . k_0."""
+    q = _rand((2, 3, 1, 16), 3)
+    k = _rand((2, 3, 1, 16), 4)
+    v = _rand((2, 3, 1, 16), 5)
+    for causal in (False, True):
+        o, lse = _run(lib, q, k, v, 0.3, causal)
+        np.testing.assert_array_equal(o, v.astype(np.float64))
+        want = 0.3 * np.einsum("bhnd,bhnd->bhn", q.astype(np.float64), k.astype(np.float64))
+        np.testing.assert_allclose(lse, want, rtol=0, atol=1e-13)
+
+
+def pin_causal_row0(lib):
+    """Causal row 0 sees only key 0: O_0 = V_0 exactly, lse_0 = scale * q_0 . k_0."""
+    q = _rand((1, 2, 50, 32), 6, 3.0)
+    k = _rand((1, 2, 50, 32), 7)
+    v = _rand((1, 2, 50, 32), 8)
+    o, lse = _run(lib, q, k, v, 0.25, True)
+    np.testing.assert_array_equal(o[:, :, 0], v[:, :, 0].astype(np.float64))
+    want = 0.25 * (q[:, :, 0].astype(np.float64) * k[:, :, 0].astype(np.float64)).sum(-1)
+    np.testing.assert_allclose(lse[:, :, 0], want, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- invariances
+
+def pin_affine_v(lib):
+    """Softmax weights sum to 1, so O(a V + b) = a O(V) + b (b a constant row)."""
+    q = _rand((1, 2, 40, 8), 9, 2.0)
+    k = _rand((1, 2, 40, 8), 10)
+    v = _rand((1, 2, 40, 8), 11)
+    a, bvec = 0.5, np.linspace(-2, 2, 8).astype(np.float32)
+    v2 = (a * v + bvec).astype(np.float32)  # exact: a is a power of two... up to fp32 add
+    for causal in (False, True):
+        o1, l1 = _run(lib, q, k, v, 0.4, causal)
+        o2, l2 = _run(lib, q, k, v2, 0.4, causal)
+        # reference through the fp32 values actually passed
+        ones = np.ones_like(v)
+        o_one, _ = _run(lib, q, k, ones, 0.4, causal)
+        np.testing.assert_allclose(o_one, 1.0, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(o2, a * o1 + bvec, rtol=0, atol=1e-6)
+        np.testing.assert_array_equal(l1, l2)
+
+
+def pin_key_permutation(lib):
+    """Non-causal attention is a sum over keys: permuting K and V rows together
+    changes nothing."""
+    q = _rand((1, 1, 33, 16), 12, 2.0)
+    k = _rand((1, 1, 33, 16), 13)
+    v = _rand((1, 1, 33, 16), 14)
+    perm = np.random.default_rng(15).permutation(33)
+    o1, l1 = _run(lib, q, k, v, 0.5, False)
+    o2, l2 = _run(lib, q, k[:, :, perm], v[:, :, perm], 0.5, False)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+def pin_future_keys_ignored(lib):
+    """Causal row i must not depend on keys/values after i."""
+    q = _rand((1, 1, 30, 8), 16, 2.0)
+    k = _rand((1, 1, 30, 8), 17)
+    v = _rand((1, 1, 30, 8), 18)
+    o1, l1 = _run(lib, q, k, v, 0.6, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 20:] = 100.0
+    v2[:, :, 20:] = -50.0
+    o2, l2 = _run(lib, q, k2, v2, 0.6, True)
+    np.testing.assert_array_equal(o1[:, :, :20], o2[:, :, :20])
+    np.testing.assert_array_equal(l1[:, :, :20], l2[:, :, :20])
+    assert np.abs(o1[:, :, 20:] - o2[:, :, 20:]).max() > 1.0
+
+
+def pin_softmax_shift(lib):
+    """Adding one vector w to every key adds scale*q_i.w to every score of row i:
+    O is unchanged and lse_i moves by exactly that amount."""
+    q = _rand((1, 2, 24, 8), 19)
+    k = _rand((1, 2, 24, 8), 20)
+    v = _rand((1, 2, 24, 8), 21)
+    w = np.array([0.5, -1.0, 0.25, 2.0, 0.0, -0.5, 1.0, 0.125], np.float32)
+    k2 = (k + w).astype(np.float32)
+    for causal in (False, True):
+        o1, l1 = _run(lib, q, k, v, 0.8, causal)
+        o2, l2 = _run(lib, q, k2, v, 0.8, causal)
+        # fp32 rounding of k + w perturbs scores by ~1e-7; compare at that level
+        np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-5)
+        shift = 0.8 * (q.astype(np.float64) @ w.astype(np.float64))
+        np.testing.assert_allclose(l2 - l1, shift, rtol=0, atol=1e-5)
+
+
+def pin_lse_bounds(lib):
+    """max_j s_ij <= lse_i <= max_j s_ij + ln(#allowed keys)."""
+    q = _rand((1, 1, 64, 16), 22, 3.0)
+    k = _rand((1, 1, 64, 16), 23)
+    v = _rand((1, 1, 64, 16), 24)
+    s = 0.5 * (q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T)
+    for causal in (False, True):
+        _, lse = _run(lib, q, k, v, 0.5, causal)
+        for i in range(64):
+            allowed = s[i, : i + 1] if causal else s[i]
+            assert allowed.max() - 1e-12 <= lse[0, 0, i] <= allowed.max() + math.log(len(allowed)) + 1e-12
+
+
+def pin_row_subset(lib):
+    """Asking for a subset of rows returns exactly those rows of the full run."""
+    q = _rand((2, 2, 70, 8), 25)
+    k = _rand((2, 2, 70, 8), 26)
+    v = _rand((2, 2, 70, 8), 27)
+    rows = np.array([[[0, 5, 69], [1, 2, 3]], [[68, 0, 30], [7, 7, 7]]], np.int64)
+    for causal in (False, True):
+        of, lf = _run(lib, q, k, v, 0.3, causal)
+        os_, ls = _run(lib, q, k, v, 0.3, causal, rows=rows)
+        for b in range(2):
+            for h in range(2):
+                np.testing.assert_array_equal(os_[b, h], of[b, h, rows[b, h]])
+                np.testing.assert_array_equal(ls[b, h], lf[b, h, rows[b, h]])
+
+
+# ---------------------------------------------------------------- online ledger (pages)
+
+def online_ledger(scores, values, tile, rescale=True):
+    """The tile-by-tile ledger of FlashAttention, Playable (EP 04): a running max m,
+    a running sum l and a rescale of everything accumulated whenever a tile
+    brings a bigger max.  With ``rescale=False`` it is the naive streamer that
+    the page shows going wrong."""
+    m, l = -math.inf, 0.0
+    acc = np.zeros(values.shape[1])
+    for t0 in range(0, len(scores), tile):
+        s = scores[t0:t0 + tile]
+        m_new = max(m, float(s.max()))
+        r = math.exp(m - m_new) if (rescale and m != -math.inf) else 1.0
+        e = np.exp(s - m_new)
+        l = l * r + float(e.sum())
+        acc = acc * r + e @ values[t0:t0 + tile]
+        m = m_new
+    return acc / l, m + math.log(l)
+
+
+def pin_online_ledger(lib):
+    """Online softmax equals the all-at-once softmax (the page claims agreement
+    to 15 decimals); rows are built so that later tiles bring larger maxima."""
+    N, d = 96, 4
+    rng = np.random.default_rng(28)
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[0, 0, :, 0] = 1.0
+    k = np.zeros((1, 1, N, d), np.float32)
+    # increasing trend + noise: the running max keeps growing across tiles
+    k[0, 0, :, 0] = (np.linspace(0, 12, N) + rng.standard_normal(N)).astype(np.float32)
+    v = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    o, lse = _run(lib, q, k, v, 1.0, False)
+    scores = k[0, 0, :, 0].astype(np.float64)
+    for tile in (1, 3, 64):
+        o_led, lse_led = online_ledger(scores, v[0, 0].astype(np.float64), tile)
+        np.testing.assert_allclose(o[0, 0, 0], o_led, rtol=0, atol=1e-13)
+        assert abs(lse[0, 0, 0] - lse_led) < 1e-13
+
+
+def check_no_rescale_fails():
+    """Negative control (EP 04): the streamer without rescale is far off on the
+    same row, so the ledger comparison above has teeth."""
+    N, d = 96, 4
+    rng = np.random.default_rng(28)
+    scores = rng.standard_normal(N)
+    scores[-8:] += 4.0  # the last tile brings a bigger max
+    values = rng.standard_normal((N, d))
+    values[:-8] += 1.0
+    values[-8:] -= 1.0
+    good, _ = online_ledger(scores, values, 8)
+    bad, _ = online_ledger(scores, values, 8, rescale=False)
+    return float(np.abs(bad - good).max() / np.abs(good).max())
+
+
+# ---------------------------------------------------------------- library cross-check
+
+def pin_torch_sdpa(lib):
+    """torch's fp64 math attention and logsumexp agree with the oracle."""
+    for (B, H, N, d, causal, seed) in [(1, 2, 65, 16, False, 29), (2, 1, 130, 32, True, 30),
+                                        (1, 1, 257, 64, True, 31)]:
+        q = _rand((B, H, N, d), seed, 2.0)
+        k = _rand((B, H, N, d), seed + 100)
+        v = _rand((B, H, N, d), seed + 200)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = _run(lib, q, k, v, scale, causal)
+        qt, kt, vt = (torch.from_numpy(x).double() for x in (q, k, v))
+        ot = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal, scale=scale)
+        s = scale * qt @ kt.transpose(-1, -2)
+        if causal:
+            s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+        lt = torch.logsumexp(s, dim=-1)
+        np.testing.assert_allclose(o, ot.numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lt.numpy(), rtol=0, atol=1e-12)
+
+
+ALL_PINS = [
+    pin_hand_worked, pin_q_zero_mean_of_v, pin_single_key, pin_causal_row0, pin_affine_v,
+    pin_key_permutation, pin_future_keys_ignored, pin_softmax_shift, pin_lse_bounds,
+    pin_row_subset, pin_online_ledger, pin_torch_sdpa,
+]
