@@ -1,0 +1,111 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library.
+ *
+ * The operation is the one the pages state as the attention problem and then
+ * compute tile by tile:
+ *
+ *     S = scale * Q K^T,   P = softmax(S),   O = P V
+ *
+ * (Chapter 15 -- FlashAttention, "Standard vs Flash Attention": S = Q @ K^T,
+ * P = softmax(S), O = P @ V; the FlashAttention column computes the same O
+ * from tiles with an online softmax, writing O once.)  The library computes
+ * it without ever writing the N x N score matrix to memory, using the online
+ * softmax (running row max m, running row sum l, rescale of the accumulator
+ * when the max grows; FlashAttention, Playable, EP 04) and writes O and the
+ * per-row log-sum-exp exactly once (FlashAttention: Tiled & Fused, diagram:
+ * "Output O written once", with the "online-softmax stats").
+ *
+ * Not on the pages, and fixed here: the softmax scale multiplies Q K^T before
+ * the softmax; the optional causal mask keeps keys j <= i for query row i;
+ * lse_i = ln(sum_j exp(scale * q_i . k_j)) over the allowed keys (natural
+ * log, fp32).
+ *
+ * Every function is callable from C.  Pointers named "device" must point to
+ * memory of the current CUDA device; nothing here allocates or frees the
+ * caller's buffers.
+ */
+#ifndef FA_B200_FA_H
+#define FA_B200_FA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_VERSION_MAJOR 1
+#define FA_VERSION_MINOR 0
+#define FA_VERSION_PATCH 0
+
+/* Element type of q, k, v and o. */
+typedef enum {
+    FA_DTYPE_F32 = 0,  /* fp32 in, fp32 out; CUDA-core FFMA kernel */
+    FA_DTYPE_BF16 = 1  /* bf16 in, bf16 out, fp32 accumulation; tensor-core kernel */
+} fa_dtype_t;
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size, alignment, aliasing, dtype or scale */
+    FA_ERR_UNSUPPORTED = 2,      /* well-formed but not implemented (head dim other than 64/128) */
+    FA_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed; see fa_last_error() */
+    FA_ERR_DEVICE_TIMEOUT = 4    /* a kernel gave up on a bounded wait (reported by fa_check_device_status) */
+} fa_status_t;
+
+/*
+ * fa_fwd -- exact attention forward.
+ *
+ *   q, k, v  device, contiguous row-major [B][H][N][d] of `dtype` (each head's
+ *            N x d matrices Q, K, V as on the "Standard vs Flash Attention"
+ *            panel).  16-byte aligned.
+ *   o        device, [B][H][N][d] of `dtype`, written once per row.  16-byte
+ *            aligned; must not overlap q, k, v or lse.
+ *   lse      device, [B][H][N] fp32, natural-log log-sum-exp of each row's
+ *            scaled, masked scores.  4-byte aligned; must not overlap the others.
+ *   B, H, N  batch, heads, sequence length; each >= 1.  Any N is accepted (no
+ *            multiple-of-tile requirement).
+ *   d        head dimension: 64 or 128 (others: FA_ERR_UNSUPPORTED).
+ *   scale    any finite float; multiplies Q K^T before the softmax (use
+ *            1/sqrt(d) for the usual attention).
+ *   causal   0: every key is visible; non-zero: query row i sees keys j <= i.
+ *   dtype    FA_DTYPE_BF16 or FA_DTYPE_F32.
+ *   stream   a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Asynchronous: the work is enqueued on `stream` and the call returns; the
+ * buffers must stay valid until the stream reaches it.  Argument errors are
+ * reported synchronously before any CUDA call is made, and then nothing is
+ * enqueued.  A device-side timeout (a bounded wait that expired) is not seen
+ * here; call fa_check_device_status after the stream has run.
+ * Thread safety: concurrent calls from several host threads are allowed.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int64_t B, int64_t H, int64_t N, int64_t d,
+           float scale, int causal, int dtype, void* stream);
+
+/*
+ * fa_check_device_status -- synchronise `stream`, then read and clear the
+ * library's device status word for the current device.  Returns FA_OK,
+ * FA_ERR_DEVICE_TIMEOUT when a kernel launched by this library gave up on a
+ * bounded wait since the last check (its outputs are then invalid), or
+ * FA_ERR_CUDA.
+ */
+int fa_check_device_status(void* stream);
+
+/* fa_status_string -- static, never-NULL description of a status code. */
+const char* fa_status_string(int status);
+
+/*
+ * fa_last_error -- description of the last failure seen by the calling host
+ * thread (which argument was rejected, or the CUDA error text).  The pointer
+ * stays valid until the thread's next call into the library.
+ */
+const char* fa_last_error(void);
+
+/* fa_version -- MAJOR * 10000 + MINOR * 100 + PATCH of the loaded library. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H */

@@ -1,0 +1,108 @@
+"""The C-ABI boundary on the CPU: the library loads without a GPU, exports every
+entry point include/fa.h declares, and rejects bad arguments before making
+any CUDA call (so these run, and must pass, on a machine with no GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import tiled_exact_attention_fa_b200 as fa
+from tiled_exact_attention_fa_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", h) for h in os.listdir(os.path.join(ROOT, "include")) if h.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.library()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(fa_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa_fwd", "fa_check_device_status", "fa_status_string", "fa_last_error", "fa_version"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\S+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        getattr(lib, name)  # and ctypes can resolve it
+
+
+def test_binding_covers_every_entry_point():
+    assert set(declared_functions()) == set(fa._SIGNATURES)
+
+
+def test_version(lib):
+    assert fa.version() == 10000
+
+
+def test_status_strings(lib):
+    for code in range(0, 5):
+        s = lib.fa_status_string(code).decode()
+        assert s.startswith(("FA_OK", "FA_ERR_"))
+    assert "unknown" in lib.fa_status_string(99).decode()
+
+
+# Fake, never-dereferenced addresses: every case below must be rejected by
+# the argument checks, which run before any CUDA call.
+A = 0x10000000
+NB = 1 << 24  # spacing between the fake buffers
+
+
+def call(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,
+         scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, None)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(k=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(v=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(o=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(lse=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(B=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(H=-1), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(N=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(d=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(dtype=7), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(q=A + 8), fa.FA_ERR_INVALID_ARGUMENT),          # misaligned
+    (dict(o=A + 3 * NB + 2), fa.FA_ERR_INVALID_ARGUMENT),  # misaligned
+    (dict(lse=A + 4 * NB + 2), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(o=A + 16), fa.FA_ERR_INVALID_ARGUMENT),          # o overlaps q
+    (dict(lse=A + 3 * NB + 64), fa.FA_ERR_INVALID_ARGUMENT),  # lse inside o
+    (dict(N=(1 << 30) + 1), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(B=1 << 20, H=1 << 20), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+])
+def test_rejected_before_cuda(lib, kwargs, code):
+    lib.fa_fwd.restype = ctypes.c_int
+    assert call(lib, **kwargs) == code
+    assert lib.fa_last_error().decode() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_no_gpu_is_an_error_not_a_fallback(lib):
+    # well-formed arguments on a machine without a GPU: a CUDA error, never a result
+    assert call(lib) == fa.FA_ERR_CUDA
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises((RuntimeError, AssertionError)):
+        fa.forward(q, q, q)

@@ -1,0 +1,164 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Outputs are NaN-filled before each call (an unwritten row fails), and guard
+bands around O and lse must come back untouched.  Every input is seeded.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_exact_attention_fa_b200 as fa
+from tiled_exact_attention_fa_b200 import build as fa_build
+from tiled_exact_attention_fa_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096  # elements on each side of O and lse (keeps 16-byte alignment)
+SENTINEL = 4096.0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    fa_build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    fa.library()
+
+
+def run_guarded(q, k, v, scale, causal, stream=None):
+    """fa_fwd through the C ABI into NaN-filled, guard-banded outputs on the GPU."""
+    B, H, N, d = q.shape
+    n_o, n_l = q.numel(), B * H * N
+    o_buf = torch.full((n_o + 2 * GUARD,), SENTINEL, dtype=q.dtype, device=q.device)
+    l_buf = torch.full((n_l + 2 * GUARD,), SENTINEL, dtype=torch.float32, device=q.device)
+    o = o_buf[GUARD:GUARD + n_o].view(B, H, N, d)
+    lse = l_buf[GUARD:GUARD + n_l].view(B, H, N)
+    o.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    fa.forward_into(q, k, v, o, lse, scale=scale, causal=causal, stream=stream)
+    fa.check_device_status(stream)
+    for buf, n in ((o_buf, n_o), (l_buf, n_l)):
+        assert bool((buf[:GUARD] == SENTINEL).all()) and bool((buf[GUARD + n:] == SENTINEL).all()), \
+            "write outside the output buffer"
+    return o, lse
+
+
+def check_against_oracle(q, k, v, scale, causal, rows=None, strict_raw=True):
+    o, lse = run_guarded(q.cuda(), k.cuda(), v.cuda(), scale, causal)
+    o_ref, lse_ref = parity.oracle_reference(q, k, v, scale, causal, rows)
+    o, lse = o.cpu(), lse.cpu()
+    if rows is not None:
+        o, lse = parity.gather_rows(o, rows), parity.gather_rows(lse, rows)
+    return parity.compare(o, lse, o_ref, lse_ref, q.dtype, strict_raw=strict_raw), o, lse
+
+
+# ------------------------------------------------------------ small and ragged shapes
+
+def test_first_small_bf16():
+    q, k, v = W.random_qkv(1, 2, 256, 128, torch.bfloat16, seed=11)
+    for causal in (False, True):
+        check_against_oracle(q, k, v, 1 / math.sqrt(128), causal)
+
+
+EDGE_N = [1, 2, 127, 128, 129, 200, 255, 256, 257, 383, 384, 511, 640]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", EDGE_N)
+def test_bf16_edge_shapes(N, d, causal):
+    q, k, v = W.random_qkv(1, 3, N, d, torch.bfloat16, seed=100 + N + d)
+    check_against_oracle(q, k, v, 1 / math.sqrt(d), causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 31, 33, 100, 256])
+def test_f32_edge_shapes(N, d, causal):
+    q, k, v = W.random_qkv(2, 2, N, d, torch.float32, seed=300 + N + d)
+    check_against_oracle(q, k, v, 1 / math.sqrt(d), causal)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("scale", [-0.3, 0.0, 1.0])
+def test_scale_values(scale, dtype):
+    q, k, v = W.random_qkv(1, 2, 300, 64, dtype, seed=17)
+    for causal in (False, True):
+        check_against_oracle(q, k, v, scale, causal)
+
+
+def test_many_units_per_cta():
+    # 4*40 heads x 2 query blocks = 320 work units: several per persistent CTA
+    q, k, v = W.random_qkv(4, 40, 512, 128, torch.bfloat16, seed=19)
+    rows = torch.arange(0, 512, 7, dtype=torch.int64).expand(4, 40, -1).contiguous()
+    for causal in (False, True):
+        check_against_oracle(q, k, v, 1 / math.sqrt(128), causal, rows=rows)
+
+
+def test_wide_score_range_rescales():
+    # Q scaled by 8 with increasing keys: the running max keeps growing
+    q, k, v = W.random_qkv(1, 2, 1024, 128, torch.bfloat16, seed=23, q_mult=8.0)
+    ramp = torch.linspace(0, 3, 1024).view(1, 1, 1024, 1)
+    k = (k.float() + ramp).to(torch.bfloat16)
+    for causal in (False, True):
+        check_against_oracle(q, k, v, 1 / math.sqrt(128), causal, strict_raw=False)
+
+
+# ------------------------------------------------------------ behaviour
+
+def test_deterministic_and_stream():
+    q, k, v = (x.cuda() for x in W.random_qkv(2, 4, 1000, 128, torch.bfloat16, seed=29))
+    o1, l1 = run_guarded(q, k, v, 0.1, True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o2, l2 = run_guarded(q, k, v, 0.1, True, stream=s)
+    s.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_causal_row0_is_exact():
+    # causal row 0 sees only key 0: P = 1 exactly, so O_0 = V_0 bit for bit
+    q, k, v = (x.cuda() for x in W.random_qkv(2, 3, 700, 128, torch.bfloat16, seed=31))
+    o, lse = run_guarded(q, k, v, 1 / math.sqrt(128), True)
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
+    want = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) / math.sqrt(128)
+    assert float((lse[:, :, 0].double() - want).abs().max()) < 1e-4
+
+
+def test_host_tensors_round_trip():
+    q, k, v = W.random_qkv(1, 2, 384, 64, torch.bfloat16, seed=37)
+    o, lse = fa.forward(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True)
+    assert not o.is_cuda and not lse.is_cuda
+    o_ref, lse_ref = parity.oracle_reference(q, k, v, 1 / math.sqrt(64), True)
+    parity.compare(o, lse, o_ref, lse_ref, torch.bfloat16)
+
+
+def test_invalid_arguments_on_gpu():
+    q = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 1, 64, device="cuda")
+    with pytest.raises(fa.FaError) as e:
+        fa.forward_into(q, q, q, q, lse)  # o aliases q
+    assert e.value.status == fa.FA_ERR_INVALID_ARGUMENT
+    big = torch.zeros(1, 1, 64, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FaError) as e:
+        fa.forward(big, big, big)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+    fa.forward_into(q, q, q, o, lse)  # still usable after rejected calls
+    fa.check_device_status()
+
+
+# ------------------------------------------------------------ the five workloads
+
+@pytest.mark.parametrize("w", W.WORKLOADS, ids=[w.name for w in W.WORKLOADS])
+def test_workload(w):
+    q, k, v = W.make_inputs(w)
+    rows = None if w.sample_rows is None else W.sample_rows(w)
+    stats, o, _ = check_against_oracle(q, k, v, w.scale, w.causal, rows=rows,
+                                       strict_raw=(w.q_mult == 1.0))
+    print(w.name, stats)
+    if w.causal:
+        # row 0 of every head (always among the checked rows, first after sorting): exact
+        assert torch.equal(o[:, :, 0], v[:, :, 0])

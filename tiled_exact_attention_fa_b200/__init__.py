@@ -1,0 +1,140 @@
+"""B200 (sm_100a) exact attention forward: O = softmax(scale * Q K^T [causal]) V.
+
+The compute runs in libfa_b200.so (hand-written CUDA for sm_100a behind the C
+ABI in include/fa.h).  This module only marshals arguments to it: torch is
+used for device memory and the current stream, nothing else.  There is no
+fallback: if the library is missing or the GPU is not an sm_100 part, calls
+raise.
+
+    import tiled_exact_attention_fa_b200 as fa
+    o, lse = fa.forward(q, k, v, causal=True)      # q, k, v: [B, H, N, d]
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
+
+FA_DTYPE_F32 = 0
+FA_DTYPE_BF16 = 1
+FA_OK = 0
+FA_ERR_INVALID_ARGUMENT = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_DEVICE_TIMEOUT = 4
+
+# Every entry point of include/fa.h with its ctypes signature.
+_SIGNATURES = {
+    "fa_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
+               [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fa_last_error": (ctypes.c_char_p, []),
+    "fa_version": (ctypes.c_int, []),
+}
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, detail: str = ""):
+        self.status = status
+        msg = library().fa_status_string(status).decode()
+        super().__init__(f"{msg}{': ' + detail if detail else ''}")
+
+
+def library() -> ctypes.CDLL:
+    """The loaded C-ABI library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m tiled_exact_attention_fa_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def version() -> int:
+    return int(library().fa_version())
+
+
+def _check(status: int):
+    if status != FA_OK:
+        raise FaError(status, library().fa_last_error().decode())
+
+
+_DTYPES = {torch.bfloat16: FA_DTYPE_BF16, torch.float32: FA_DTYPE_F32}
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, stream) -> int:
+    """Direct C-ABI call with raw device pointers (ints); returns the status code."""
+    return int(library().fa_fwd(q, k, v, o, lse, B, H, N, d, scale, int(causal), dtype, stream))
+
+
+def forward_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                 lse: torch.Tensor, *, scale: float | None = None, causal: bool = False,
+                 stream: torch.cuda.Stream | None = None) -> None:
+    """Run the forward into caller-provided CUDA tensors o [B,H,N,d] and lse [B,H,N] fp32."""
+    if q.dtype not in _DTYPES or not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise TypeError("q, k, v, o must all be bf16 or all fp32")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be fp32")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
+        raise ValueError("q, k, v, o must share one [B, H, N, d] shape")
+    if lse.shape != q.shape[:3]:
+        raise ValueError("lse must be [B, H, N]")
+    for t in (q, k, v, o, lse):
+        if not t.is_cuda:
+            raise ValueError("forward_into needs CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    with torch.cuda.device(q.device):
+        _check(fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, float(scale), causal, _DTYPES[q.dtype], s))
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
+            causal: bool = False):
+    """Exact attention forward.  Returns (o, lse).
+
+    q, k, v: [B, H, N, d] bf16 or fp32, d in {64, 128}.  CUDA tensors give CUDA
+    outputs.  Host tensors are copied to the current CUDA device (pinned memory
+    makes the copies asynchronous), computed there, and the outputs are copied
+    back into host tensors: the host-to-host path through the same kernels.
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v = (x.to(dev, non_blocking=True) for x in (q, k, v))
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    forward_into(q, k, v, o, lse, scale=scale, causal=causal)
+    if host:
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return o_h, lse_h
+    return o, lse
+
+
+def check_device_status(stream: torch.cuda.Stream | None = None) -> None:
+    """Synchronise and raise FaError(FA_ERR_DEVICE_TIMEOUT) if a kernel gave up on a wait."""
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(int(library().fa_check_device_status(s)))

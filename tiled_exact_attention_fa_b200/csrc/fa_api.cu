@@ -1,0 +1,235 @@
+// fa_api.cu -- the C ABI (include/fa.h): argument checks, kernel choice,
+// TMA tensor-map encoding, persistent-grid sizing and launch on the caller's
+// stream.  All compute runs in the kernels of fa_fwd_tc.cuh (bf16, tensor
+// cores) and fa_fwd_simt.cuh (fp32, CUDA cores).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "fa.h"
+#include "fa_fwd_simt.cuh"
+#include "fa_fwd_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(FA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorName(e) + " (" +
+                                 cudaGetErrorString(e) + ")");
+}
+
+// Per-device state created on the first call that runs on that device: the
+// 16-byte device status word written by kernels that give up on a bounded
+// wait, the SM count for the persistent grid, and whether the kernels' shared
+// memory limits were raised.  Kept until process exit.
+struct DeviceState {
+    bool ready = false;
+    int* status = nullptr;
+    int sm_count = 0;
+    int cc_major = 0;
+    bool smem_raised[4] = {false, false, false, false};
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_state(DeviceState** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& s = g_dev[dev];
+    if (!s.ready) {
+        if ((e = cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+        if ((e = cudaDeviceGetAttribute(&s.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute(compute capability)");
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void* fn = nullptr;
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+                return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        if ((e = cudaMalloc(&s.status, 16)) != cudaSuccess) return cuda_fail(e, "cudaMalloc(status word)");
+        if ((e = cudaMemset(s.status, 0, 16)) != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
+        s.ready = true;
+    }
+    *out = &s;
+    return FA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// 3-D view (d, N, B*H) of a [B*H][N][d] bf16 tensor, boxes of 64 x 128 x 1
+// with 128-byte swizzle; rows past N read as zeros.
+int encode_tile_map(CUtensorMap* map, const void* ptr, int64_t bh, int64_t n, int64_t d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(n * d * 2)};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fa::tc::kBlockM), 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                          elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
+    return FA_OK;
+}
+
+template <int D, bool kCausal>
+int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const void* v, void* o, float* lse,
+                int64_t bh, int64_t n, float scale, cudaStream_t stream) {
+    using L = fa::tc::Layout<D>;
+    auto kernel = fa::tc::fa_fwd_bf16_kernel<D, kCausal>;
+    if (!st->smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->smem_raised[slot] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+
+    fa::tc::Params p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.status = st->status;
+    p.bh = static_cast<int>(bh);
+    p.n = static_cast<int>(n);
+    p.num_qblocks = static_cast<int>((n + fa::tc::kUnitRows - 1) / fa::tc::kUnitRows);
+    p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
+    p.num_units = p.bh * p.num_qblocks;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
+    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the bf16 attention kernel");
+    return FA_OK;
+}
+
+template <int D, bool kCausal>
+int launch_f32(const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh, int64_t n,
+               float scale, cudaStream_t stream) {
+    fa::simt::Params p;
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.o = static_cast<float*>(o);
+    p.lse = lse;
+    p.n = static_cast<int>(n);
+    p.scale = scale;
+    dim3 grid(static_cast<unsigned>((n + fa::simt::kRows - 1) / fa::simt::kRows), static_cast<unsigned>(bh));
+    fa::simt::fa_fwd_f32_kernel<D, kCausal><<<grid, fa::simt::kThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the fp32 attention kernel");
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return FA_VERSION_MAJOR * 10000 + FA_VERSION_MINOR * 100 + FA_VERSION_PATCH; }
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK: success";
+        case FA_ERR_INVALID_ARGUMENT: return "FA_ERR_INVALID_ARGUMENT: bad pointer, size, alignment, aliasing, dtype or scale";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: well-formed request this library does not implement";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+        case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait; outputs invalid";
+        default: return "unknown fa status code";
+    }
+}
+
+const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t N,
+           int64_t d, float scale, int causal, int dtype, void* stream) {
+    g_last_error.clear();
+    // ---- argument checks: all before any CUDA call
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    const int64_t bh = B * H;
+    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
+    const int64_t units = bh * ((N + 255) / 256);
+    if (units > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
+    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
+    if (bh > (int64_t{1} << 62) / (N * d * elem)) return fail(FA_ERR_INVALID_ARGUMENT, "tensor size overflows");
+    const size_t tensor_bytes = static_cast<size_t>(bh * N * d * elem);
+    const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
+    auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16))
+        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+    if (misaligned(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
+        overlaps(o, tensor_bytes, v, tensor_bytes) || overlaps(o, tensor_bytes, lse, lse_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
+    if (overlaps(lse, lse_bytes, q, tensor_bytes) || overlaps(lse, lse_bytes, k, tensor_bytes) ||
+        overlaps(lse, lse_bytes, v, tensor_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
+
+    // ---- device set-up (first call per device) and dispatch
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool c = causal != 0;
+    if (dtype == FA_DTYPE_BF16) {
+        if (st->cc_major != 10)
+            return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
+        if (d == 128) return c ? launch_bf16<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
+                               : launch_bf16<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
+        return c ? launch_bf16<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
+                 : launch_bf16<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
+    }
+    if (d == 128) return c ? launch_f32<128, true>(q, k, v, o, lse, bh, N, scale, s)
+                           : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
+    return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
+             : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+}
+
+int fa_check_device_status(void* stream) {
+    g_last_error.clear();
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int h = 0;
+    if ((e = cudaMemcpy(&h, st->status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpy(status word)");
+    if (h != 0) {
+        if ((e = cudaMemset(st->status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
+        return fail(FA_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait");
+    }
+    return FA_OK;
+}
+
+}  // extern "C"
