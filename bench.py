@@ -1,0 +1,330 @@
+#!/usr/bin/env python
+"""Benchmark of the exact attention forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one fa_fwd call over the whole workload (default: bf16, B=2, H=32,
+N=8192, d=128, causal): the tiles of Q, K, V streamed through the fused kernel
+and O plus the log-sum-exp written once.  The metric is attention TFLOP/s
+(4*B*H*N^2*d, halved for causal) with inputs resident in HBM; the same metric
+end to end (host buffers in, host buffers out, copies included) is reported as
+`e2e`.  Under torchrun every rank runs its own batch of the workload on its own
+GPU (weak scaling, no collective on the data path); the job's time is the
+slowest rank's.
+
+`--impl reference` times the fp64 CPU oracle (test infrastructure, the
+deliberately slow plain definition) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tiled_exact_attention_fa_b200 import accounting  # noqa: E402
+from tiled_exact_attention_fa_b200 import dist as fdist  # noqa: E402
+from tiled_exact_attention_fa_b200 import workloads as W  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (bf16, d=128, N=8K causal) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2**20
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--legs", default="kernel,e2e,cpu",
+                    help="comma list of kernel,e2e,cpu (profiling runs use --legs kernel)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def kernel_digest() -> str:
+    from tiled_exact_attention_fa_b200 import build as fb
+    return fb._inputs_digest()
+
+
+def traffic_from_profile(w: W.Workload):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel changed since."""
+    path = os.path.join(PROFILE_DIR, f"traffic_{w.name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_digest") != kernel_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.gpu = gpu_index
+        self.enabled = enabled
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        if not self.enabled:
+            return self
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), util=float(parts[4]),
+                                     reasons=[n for n, v in zip(["hw_slowdown", "hw_thermal_slowdown",
+                                                                  "sw_thermal_slowdown", "sw_power_cap"],
+                                                                 parts[5:]) if v.lower() == "active"]))
+                except ValueError:
+                    continue
+        os.unlink(self.file.name)
+        loaded = [r for r in rows if r["util"] >= 50] or rows
+        if not loaded:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        reasons = sorted({x for r in loaded for x in r["reasons"]})
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": loaded[0]["smax"],
+                "reasons": reasons, "samples": len(loaded)}
+
+
+def sample_rows_for(w: W.Workload, seconds: float, seed: int):
+    """A bounded random sample of (head, row) pairs whose oracle time is about
+    `seconds` on this host; returns (rows [1, h, R], head slice, work in FLOP)."""
+    import numpy as np
+    import oracle
+    g = torch.Generator().manual_seed(seed)
+    heads = min(w.B * w.H, max(1, oracle.num_threads() // 2))
+    shape = (1, heads, w.N, w.d)
+
+    def draw():
+        x = torch.randn(shape, generator=g)
+        return x.to(w.dtype).float().numpy()
+
+    q, k, v = draw(), draw(), draw()
+    if w.q_mult != 1.0:
+        q = q * w.q_mult
+    rng = np.random.default_rng(seed)
+
+    def run(R):
+        rows = np.sort(rng.integers(0, w.N, size=(1, heads, R)), axis=-1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_fwd(q, k, v, w.scale, w.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        keys = (rows + 1) if w.causal else np.full_like(rows, w.N)
+        return dt, float((4.0 * w.d * keys).sum()), rows
+
+    dt, work, _ = run(8)
+    rate = work / max(dt, 1e-6)
+    per_row = 4.0 * w.d * (w.N / 2 if w.causal else w.N)
+    R = int(max(8, min(w.N, seconds * rate / per_row / heads)))
+    return (q, k, v), heads, R, run
+
+
+def cpu_leg(w: W.Workload, seconds: float):
+    import oracle
+    _, heads, R, run = sample_rows_for(w, seconds, seed=w.seed + 7)
+    dt, work, _ = run(R)
+    return {"value": work / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{heads} heads x {R} random query rows of {w.name} (fp64 oracle on host cores, "
+                      f"{dt:.1f} s; work counted as 4*d per visible key)"}
+
+
+def run_reference(a, w: W.Workload):
+    rank, _, world = fdist.env_world()
+    if rank != 0:
+        return 0
+    import oracle
+    total_steps = a.steps + a.warmup
+    per_step_s = max(0.05, min(5.0, 150.0 / max(1, total_steps)))
+    _, heads, R, run = sample_rows_for(w, per_step_s, seed=w.seed + 11)
+    for _ in range(a.warmup):
+        run(R)
+    times, works = [], []
+    for _ in range(a.steps):
+        dt, work, _ = run(R)
+        times.append(dt)
+        works.append(work)
+    value = sum(works) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                                        "causal": w.causal, "seed": w.seed},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"each step: {heads} heads x {R} random query rows of {w.name}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(a, w: W.Workload):
+    import tiled_exact_attention_fa_b200 as fa
+
+    rank, local_rank, world = fdist.env_world()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        fdist.init("nccl", timeout_s=300)
+    legs = set(a.legs.split(","))
+
+    # every rank runs its own batch of the workload (independent units, weak scaling)
+    wr = W.Workload(w.name, w.dtype, w.B, w.H, w.N, w.d, w.causal, w.seed + 1000 * rank, w.q_mult)
+    q_h, k_h, v_h = W.make_inputs(wr, pin=True)
+    q, k, v = (x.to(dev, non_blocking=True) for x in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = accounting.attention_flops(w.B, w.H, w.N, w.d, w.causal)
+    in_bytes = 3 * q.numel() * q.element_size()
+    alg_bytes = accounting.algorithmic_bytes(w.B, w.H, w.N, w.d, q.element_size())
+
+    def step():
+        fa.forward_into(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+
+    for _ in range(a.warmup):
+        step()
+    fa.check_device_status()
+
+    line = {"metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if
+            w.dtype == torch.bfloat16 else "f32", "data": "synthetic"}
+    line["config"] = {
+        "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "seed": w.seed,
+        "per_rank": "own seeded batch (seed + 1000*rank), no collective on the data path",
+        "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB, no flush between steps"
+        if in_bytes > L2_BYTES else "inputs smaller than L2: not flushed (not a valid headline)",
+        "flop_per_step": flops}
+
+    elapsed_ms = None
+    if "kernel" in legs:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
+            fdist.barrier(dev)
+            torch.cuda.synchronize(dev)
+            start.record(stream)
+            for _ in range(a.steps):
+                step()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+            fdist.barrier(dev)
+        fa.check_device_status()
+        elapsed_ms = fdist.max_over_ranks(start.elapsed_time(end), dev)
+        ms = elapsed_ms / a.steps
+        tflops_rank = flops / (ms * 1e-3) / 1e12
+        peak, peak_sus, hbm, peak_kind = measured_peaks()
+        line["value"] = world * tflops_rank
+        line["ms_per_step"] = ms
+        line["pct_of_bf16_peak"] = 100.0 * tflops_rank / peak
+        line["roofline"] = {
+            "bound": "tensor", "achieved": tflops_rank, "peak": peak, "unit": "TFLOP/s",
+            "frac": tflops_rank / peak, "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
+            "frac_of_sustained": tflops_rank / peak_sus,
+            "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
+            "kernel": f"fa_fwd_bf16_kernel<{w.d},{str(w.causal).lower()}>" if w.dtype == torch.bfloat16
+            else f"fa_fwd_f32_kernel<{w.d},{str(w.causal).lower()}>",
+            "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
+        line["clocks"] = clocks.summary()
+        line["gpu_launches"] = a.steps
+
+    if "e2e" in legs:
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        fa.forward(q_h, k_h, v_h, scale=w.scale, causal=w.causal, out=(o_h, l_h))  # warm the allocator
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fdist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(a.e2e_steps):
+            fa.forward(q_h, k_h, v_h, scale=w.scale, causal=w.causal, out=(o_h, l_h))
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        fdist.barrier(dev)
+        e2e_ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.e2e_steps
+        line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": in_bytes,
+                       "d2h_bytes_per_step": o.numel() * o.element_size() + lse.numel() * 4,
+                       "api": "tiled_exact_attention_fa_b200.forward(host pinned tensors, out=host pinned)"}
+        if "value" not in line:
+            line["value"] = line["e2e"]["value"]
+
+    if "cpu" in legs and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_leg(w, a.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        fdist.barrier(dev)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    a = parse()
+    w = W.BY_NAME[a.workload]
+    if a.impl == "reference":
+        return run_reference(a, w)
+    return run_ours(a, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -162,3 +162,32 @@ def test_workload(w):
     if w.causal:
         # row 0 of every head (always among the checked rows, first after sorting): exact
         assert torch.equal(o[:, :, 0], v[:, :, 0])
+
+
+def test_queue_reuse_over_many_launches():
+    # more launches than the library has work queues: every queue is reused
+    # and must have been returned to zero by the launch before
+    q, k, v = (x.cuda() for x in W.random_qkv(1, 2, 300, 64, torch.bfloat16, seed=41))
+    o_ref, l_ref = run_guarded(q, k, v, 0.125, True)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], device="cuda")
+    for _ in range(1100):
+        fa.forward_into(q, k, v, o, lse, scale=0.125, causal=True)
+    o.fill_(float("nan"))
+    fa.forward_into(q, k, v, o, lse, scale=0.125, causal=True)
+    fa.check_device_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+
+
+def test_two_streams_interleaved():
+    q, k, v = (x.cuda() for x in W.random_qkv(2, 8, 777, 128, torch.bfloat16, seed=43))
+    ref = run_guarded(q, k, v, 0.09, False)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [(torch.empty_like(q), torch.empty(q.shape[:3], device="cuda")) for _ in range(6)]
+    for i, (o, lse) in enumerate(outs):
+        with torch.cuda.stream(streams[i % 2]):
+            fa.forward_into(q, k, v, o, lse, scale=0.09, causal=False, stream=streams[i % 2])
+    torch.cuda.synchronize()
+    fa.check_device_status()
+    for o, lse in outs:
+        assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1])

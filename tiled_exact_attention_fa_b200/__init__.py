@@ -28,7 +28,7 @@ FA_ERR_UNSUPPORTED = 2
 FA_ERR_CUDA = 3
 FA_ERR_DEVICE_TIMEOUT = 4
 
-# Every entry point of include/fa.h with its ctypes signature.
+# Every entry point of include/*.h with its ctypes signature.
 _SIGNATURES = {
     "fa_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
@@ -36,6 +36,8 @@ _SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_version": (ctypes.c_int, []),
+    # include/fa_testing.h
+    "fa_test_exp2_poly": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]),
 }
 
 _lib = None
@@ -108,13 +110,14 @@ def forward_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
 
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
-            causal: bool = False):
+            causal: bool = False, out: tuple[torch.Tensor, torch.Tensor] | None = None):
     """Exact attention forward.  Returns (o, lse).
 
     q, k, v: [B, H, N, d] bf16 or fp32, d in {64, 128}.  CUDA tensors give CUDA
     outputs.  Host tensors are copied to the current CUDA device (pinned memory
     makes the copies asynchronous), computed there, and the outputs are copied
-    back into host tensors: the host-to-host path through the same kernels.
+    back into host tensors -- `out=(o, lse)` if given (pinned, preallocated),
+    else new pinned tensors -- before the call returns.
     """
     host = not q.is_cuda
     if host:
@@ -125,12 +128,18 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float |
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     forward_into(q, k, v, o, lse, scale=scale, causal=causal)
     if host:
-        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        if out is None:
+            out = (torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                   torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True))
+        o_h, lse_h = out
         o_h.copy_(o, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
         torch.cuda.current_stream().synchronize()
         return o_h, lse_h
+    if out is not None:
+        out[0].copy_(o)
+        out[1].copy_(lse)
+        return out
     return o, lse
 
 

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -14,6 +15,7 @@
 #include <string>
 
 #include "fa.h"
+#include "fa_testing.h"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 
@@ -31,13 +33,23 @@ int cuda_fail(cudaError_t e, const char* what) {
                                  cudaGetErrorString(e) + ")");
 }
 
-// Per-device state created on the first call that runs on that device: the
-// 16-byte device status word written by kernels that give up on a bounded
-// wait, the SM count for the persistent grid, and whether the kernels' shared
-// memory limits were raised.  Kept until process exit.
+// Per-device state created on the first call that runs on that device and
+// kept until process exit: a small device workspace holding the status word
+// written by kernels that give up on a bounded wait, followed by the work
+// queues of the persistent kernel (two counters each, returned to zero by the
+// last CTA of every launch); the SM count for the persistent grid; and
+// whether the kernels' shared memory limits were raised.  Successive launches
+// take successive queues, so launches in flight at the same time (on
+// different streams) use different counters unless more than kQueues of them
+// are in flight at once.
+constexpr int kQueues = 1024;
+constexpr size_t kWorkspaceBytes = 16 + kQueues * 2 * sizeof(unsigned);
+
 struct DeviceState {
     bool ready = false;
     int* status = nullptr;
+    unsigned* queues = nullptr;
+    std::atomic<unsigned> next_queue{0};
     int sm_count = 0;
     int cc_major = 0;
     bool smem_raised[4] = {false, false, false, false};
@@ -68,8 +80,11 @@ int device_state(DeviceState** out) {
                 return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         }
-        if ((e = cudaMalloc(&s.status, 16)) != cudaSuccess) return cuda_fail(e, "cudaMalloc(status word)");
-        if ((e = cudaMemset(s.status, 0, 16)) != cudaSuccess) return cuda_fail(e, "cudaMemset(status word)");
+        void* ws = nullptr;
+        if ((e = cudaMalloc(&ws, kWorkspaceBytes)) != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+        if ((e = cudaMemset(ws, 0, kWorkspaceBytes)) != cudaSuccess) return cuda_fail(e, "cudaMemset(workspace)");
+        s.status = static_cast<int*>(ws);
+        s.queues = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + 16);
         s.ready = true;
     }
     *out = &s;
@@ -116,6 +131,7 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.status = st->status;
+    p.sched = st->queues + 2 * (st->next_queue.fetch_add(1, std::memory_order_relaxed) % kQueues);
     p.bh = static_cast<int>(bh);
     p.n = static_cast<int>(n);
     p.num_qblocks = static_cast<int>((n + fa::tc::kUnitRows - 1) / fa::tc::kUnitRows);
@@ -147,9 +163,31 @@ int launch_f32(const void* q, const void* k, const void* v, void* o, float* lse,
     return FA_OK;
 }
 
+__global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
+    const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+    float y0, y1;
+    fa::ptx::exp2_poly2(y0, y1, x0, x1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
 
 extern "C" {
+
+int fa_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+    g_last_error.clear();
+    if (n < 0 || (n > 0 && (!x || !y))) return fail(FA_ERR_INVALID_ARGUMENT, "bad exp2 test arguments");
+    if (n == 0) return FA_OK;
+    const int64_t pairs = (n + 1) / 2;
+    const unsigned blocks = static_cast<unsigned>((pairs + 255) / 256);
+    exp2_poly_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the exp2 test kernel");
+    return FA_OK;
+}
 
 int fa_version(void) { return FA_VERSION_MAJOR * 10000 + FA_VERSION_MINOR * 100 + FA_VERSION_PATCH; }
 

@@ -12,19 +12,25 @@
 // Online Softmax Enables It").
 //
 // B200 mapping (not the pages' A100/H100 sketch):
-//   * one CTA per SM, persistent over work units (b*h, 256-row query block);
-//     causal units are taken heaviest first (Chapter 15, "FlashAttention
+//   * one CTA per SM, persistent; work units (b*h, 256-row query block) are
+//     taken from a global queue in an order that keeps the units of a few
+//     heads together (their K/V stay in L2) and, under the causal mask, runs
+//     each group's heaviest query blocks first (Chapter 15, "FlashAttention
 //     Evolution": work partitioning, persistent kernels);
-//   * warp 9 is the TMA producer: Q tiles once per unit, then K_j, V_j through
-//     a ring of 128-row shared-memory slots, all 128-byte swizzled;
+//   * warp 9 is the TMA producer: it takes the next unit from the queue,
+//     publishes it to the CTA through a shared-memory ring, loads the unit's
+//     two Q tiles once and streams K_j, V_j through a ring of 128-row
+//     shared-memory slots, all 128-byte swizzled;
 //   * warp 8 issues tcgen05.mma from one thread: S_t = Q_t K_j^T into tensor
 //     memory (TMEM), then O_t += P_t V_j with P_t read from TMEM;
 //   * warps 0-3 and 4-7 are the softmax warpgroups for the unit's two query
 //     tiles (t = 0, 1), one query row per thread: they read S_t from TMEM,
 //     update m and l, write P_t (bf16) back over S_t, rescale O_t in TMEM when
-//     the max grows past a threshold, and at the end normalise O_t by l and
-//     store O and lse.  While one warpgroup exponentiates, the tensor core
-//     works on the other tile.
+//     the max grows past a threshold, and at the end normalise O_t and store
+//     O and lse.  While one warpgroup exponentiates, the tensor core works on
+//     the other tile.  Part of the exponentials run as a cubic polynomial on
+//     the FMA pipe, because at d = 128 the special-function unit alone would
+//     take as long as the tensor core.
 //   * Causal: KV blocks entirely above the diagonal are never loaded or
 //     multiplied; only the diagonal block is masked.
 //
@@ -32,7 +38,7 @@
 // O_1 at 256 + D.  P_t (bf16 pairs) occupies the first 64 columns of S_t.
 //
 // Every mbarrier wait is bounded.  On expiry the waiting thread records
-// FA_DEV_TIMEOUT in the device status word and raises a CTA-wide abort flag;
+// kDevTimeout in the device status word and raises a CTA-wide abort flag;
 // every role then leaves its loop, in-flight copies and MMAs are drained
 // (again with bounded waits) and TMEM is freed before the CTA exits.
 #pragma once
@@ -53,13 +59,16 @@ constexpr int kBlockM = 128;            // query rows per tile (one TMEM lane ea
 constexpr int kBlockN = 128;            // keys per KV block
 constexpr int kTilesPerUnit = 2;        // query tiles per work unit
 constexpr int kUnitRows = kBlockM * kTilesPerUnit;
-constexpr int kNumSoftmaxThreads = 256; // warps 0..7
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz
+constexpr int kSchedDepth = 2;              // unit ring between the producer and the other roles
+constexpr int kHeadGroup = 8;               // heads whose units are interleaved in the queue
+constexpr int kPolyPairsPer8 = 2;           // of every 8 column pairs, this many use exp2_poly2
 
 template <int D>
 struct Layout {
@@ -71,10 +80,11 @@ struct Layout {
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = kQOff + kTilesPerUnit * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
-    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 1;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base (4 B) + abort flag (4 B)
-    static constexpr int kBytes = kMiscOff + 16;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2],
+    //           sched_full[kSchedDepth], sched_empty[kSchedDepth], drain
+    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base, abort flag, unit ring
+    static constexpr int kBytes = kMiscOff + 8 + 4 * kSchedDepth;
     static constexpr int kSmemBytes = kBytes + 1024;           // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
     static constexpr uint32_t kTmemO = 256;
@@ -83,17 +93,17 @@ struct Layout {
 struct Params {
     __nv_bfloat16* o;
     float* lse;
-    int* status;
-    int bh;            // B * H
-    int n;             // sequence length
-    int num_qblocks;   // ceil(N / 256)
-    int num_kblocks;   // ceil(N / 128)
-    int num_units;     // bh * num_qblocks
-    float scale_log2;  // scale * log2(e)
+    int* status;         // device status word (kDevTimeout after a wait expired)
+    unsigned* sched;     // [0] next unit, [1] CTAs finished; both back to 0 when the launch ends
+    int bh;              // B * H
+    int n;               // sequence length
+    int num_qblocks;     // ceil(N / 256)
+    int num_kblocks;     // ceil(N / 128)
+    int num_units;       // bh * num_qblocks
+    float scale_log2;    // scale * log2(e)
 };
 
 struct Sync {
-    uint32_t bars;     // smem address of barrier 0
     volatile int* abort;
     int* status;
 };
@@ -131,17 +141,21 @@ __device__ __forceinline__ void drain_bar(const Sync& s, uint32_t bar, uint32_t 
     }
 }
 
-// Work unit -> (bh, query block).  Units of one head are consecutive so the
-// CTAs working at the same time share that head's K/V in L2; under the causal
-// mask each head's blocks go from the heaviest (last) to the lightest.
+// Queue position -> (bh, query block).  Heads go in groups of kHeadGroup;
+// inside a group the units of its heads are interleaved by query block, and
+// under the causal mask the last (heaviest) query blocks come first.
 struct Unit {
     int bh, qb;
 };
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p, bool causal) {
+    const int per_group = kHeadGroup * p.num_qblocks;
+    const int g = u / per_group;
+    const int r = u - g * per_group;
+    const int hg = min(kHeadGroup, p.bh - g * kHeadGroup);
+    const int qi = r / hg;
     Unit w;
-    w.bh = u / p.num_qblocks;
-    const int r = u - w.bh * p.num_qblocks;
-    w.qb = causal ? (p.num_qblocks - 1 - r) : r;
+    w.bh = g * kHeadGroup + (r - qi * hg);
+    w.qb = causal ? (p.num_qblocks - 1 - qi) : qi;
     return w;
 }
 
@@ -150,6 +164,51 @@ __device__ __forceinline__ int num_kv_blocks(const Params& p, int qb, int t, boo
     if (!causal) return p.num_kblocks;
     const int last = qb * (kUnitRows / kBlockN) + t;  // the diagonal block
     return min(p.num_kblocks, last + 1);
+}
+
+// One block of the online softmax for this thread's row: x_c = s_c * slv - m
+// (log2 units), p_c = 2^x_c packed to bf16 pairs, and two row sums -- in fp32
+// (for lse) and of the bf16-rounded p that enters P V (for normalising O, so
+// that O = sum(p v) / sum(p) with the same p on both sides).
+template <bool kPoly>
+__device__ __forceinline__ void exp_block(const float (&s)[kBlockN], float slv, float m_use,
+                                          uint32_t (&pk)[kBlockN / 2], float& sum, float& sum_bf16) {
+    float a[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+    float b[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    const float neg_m = -m_use;
+#pragma unroll
+    for (int pi = 0; pi < kBlockN / 2; ++pi) {
+        float x0, x1, p0, p1;
+        ptx::fma2(x0, x1, s[2 * pi], s[2 * pi + 1], slv, slv, neg_m, neg_m);
+        if (kPoly && (pi & 7) < kPolyPairsPer8) {
+            ptx::exp2_poly2(p0, p1, x0, x1);
+        } else {
+            p0 = ptx::ex2(x0);
+            p1 = ptx::ex2(x1);
+        }
+        pk[pi] = ptx::pack_bf16x2(p0, p1);
+        ptx::add2(a[pi & 3][0], a[pi & 3][1], a[pi & 3][0], a[pi & 3][1], p0, p1);
+        ptx::add_bf16x2_to_f32(b[pi & 1][0], b[pi & 1][1], pk[pi]);
+    }
+    sum = ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
+    sum_bf16 = (b[0][0] + b[0][1]) + (b[1][0] + b[1][1]);
+}
+
+// Row max (or min) of 128 values: eight independent chains of three-input ops.
+template <bool kMax>
+__device__ __forceinline__ float reduce_row(const float (&s)[kBlockN]) {
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float acc = s[16 * i];
+#pragma unroll
+        for (int c = 1; c < 15; c += 2)
+            acc = kMax ? ptx::max3(acc, s[16 * i + c], s[16 * i + c + 1])
+                       : ptx::min3(acc, s[16 * i + c], s[16 * i + c + 1]);
+        r[i] = kMax ? fmaxf(acc, s[16 * i + 15]) : fminf(acc, s[16 * i + 15]);
+    }
+    if (kMax) return fmaxf(ptx::max3(r[0], r[1], r[2]), ptx::max3(r[3], r[4], ptx::max3(r[5], r[6], r[7])));
+    return fminf(ptx::min3(r[0], r[1], r[2]), ptx::min3(r[3], r[4], ptx::min3(r[5], r[6], r[7])));
 }
 
 template <int D, bool kCausal>
@@ -175,11 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * L::kSlots + t); };
     auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * L::kSlots + t); };
     auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * L::kSlots + t); };
-    const uint32_t drain = bar0 + 8u * (10 + 2 * L::kSlots);
+    auto sched_full = [&](int i) { return bar0 + 8u * (10 + 2 * L::kSlots + i); };
+    auto sched_empty = [&](int i) { return bar0 + 8u * (10 + 2 * L::kSlots + kSchedDepth + i); };
+    const uint32_t drain = bar0 + 8u * (10 + 2 * L::kSlots + 2 * kSchedDepth);
 
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-    const Sync sync{bar0, abort_flag, p.status};
+    volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+    const Sync sync{abort_flag, p.status};
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
@@ -192,6 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < L::kSlots; ++s) {
             ptx::mbar_init(kv_full(s), 1);
             ptx::mbar_init(kv_empty(s), 1);
+        }
+        for (int i = 0; i < kSchedDepth; ++i) {
+            ptx::mbar_init(sched_full(i), 1);
+            ptx::mbar_init(sched_empty(i), 1 + kSoftmaxWarps);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -218,13 +284,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t once = ptx::policy_evict_first();  // Q: read once
             int slot = 0;
             uint32_t phase = 0;
-            // last issued phase per slot (+1), for draining on abort
+            // last issued phase per slot (+1), for draining
             uint32_t slot_issued[L::kSlots];
             uint32_t q_issued[2] = {0, 0};
             for (int s = 0; s < L::kSlots; ++s) slot_issued[s] = 0;
-            uint32_t it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++it) {
+            for (uint32_t it = 0; ok; ++it) {
+                // take the next unit from the queue and publish it to the CTA
+                const int rs = it % kSchedDepth;
+                ok = wait_bar(sync, sched_empty(rs), ((it / kSchedDepth) & 1) ^ 1);
+                if (!ok) break;
+                int u = static_cast<int>(atomicAdd(p.sched, 1u));
+                if (u >= p.num_units) u = -1;
+                unit_ring[rs] = u;
+                ptx::mbar_arrive(sched_full(rs));
+                if (u < 0) break;
+
                 const Unit w = decode_unit(u, p, kCausal);
                 const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
                 for (int t = 0; t < 2 && ok; ++t) {
@@ -260,6 +335,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (slot_issued[s]) drain_bar(sync, kv_full(s), slot_issued[s] - 1);
             for (int t = 0; t < 2; ++t)
                 if (q_issued[t]) drain_bar(sync, q_full(t), q_issued[t] - 1);
+            // The last CTA to finish returns the queue to zero for the next launch.
+            __threadfence();
+            if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+                atomicExch(p.sched, 0u);
+                atomicExch(p.sched + 1, 0u);
+            }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -270,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             int slot = 0;
             uint32_t phase = 0;
             uint32_t p_phase[2] = {0, 0};
-            uint32_t it = 0;
             bool ok = true;
 
             // S_t = Q_t K^T over the head dim: D/16 MMAs of K = 16.
@@ -305,7 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             };
 
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++it) {
+            for (uint32_t it = 0; ok; ++it) {
+                const int rs = it % kSchedDepth;
+                ok = wait_bar(sync, sched_full(rs), (it / kSchedDepth) & 1);
+                if (!ok) break;
+                const int u = unit_ring[rs];
+                ptx::mbar_arrive(sched_empty(rs));
+                if (u < 0) break;
+
                 const Unit w = decode_unit(u, p, kCausal);
                 const int n0 = num_kv_blocks(p, w.qb, 0, kCausal);
                 const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
@@ -371,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax warpgroups
-        const int t = warp >> 2;                      // query tile of this warpgroup
+        const int t = warp >> 2;                         // query tile of this warpgroup
         const int row_in_tile = (warp & 3) * 32 + lane;  // TMEM lane == tile row
         const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tmem_s = tmem + lane_addr + L::kTmemS + t * kBlockN;
@@ -380,49 +467,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
 
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        for (uint32_t it = 0; ok; ++it) {
+            const int rs = it % kSchedDepth;
+            ok = __all_sync(0xffffffffu, wait_bar(sync, sched_full(rs), (it / kSchedDepth) & 1));
+            if (!ok) break;
+            const int u = unit_ring[rs];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(sched_empty(rs));
+            if (u < 0) break;
+
             const Unit w = decode_unit(u, p, kCausal);
             const int nt = num_kv_blocks(p, w.qb, t, kCausal);
-            const int row = w.qb * kUnitRows + t * kBlockM + row_in_tile;
+            const int tile_row0 = w.qb * kUnitRows + t * kBlockM;
+            const int row = tile_row0 + row_in_tile;
             float m_run = -INFINITY;  // running max, log2 units (scale folded in)
-            float l_run = 0.f;        // running sum of 2^(x - m_run)
+            float l_run = 0.f;        // running sum of 2^(x - m_run), fp32
+            float lb_run = 0.f;       // the same sum over the bf16-rounded values
 
             for (int j = 0; j < nt; ++j) {
-                ok = wait_bar(sync, s_full(t), s_phase);
-                ok = __all_sync(0xffffffffu, ok);
+                ok = __all_sync(0xffffffffu, wait_bar(sync, s_full(t), s_phase));
                 if (!ok) break;
                 s_phase ^= 1;
                 ptx::tc_fence_after_sync();
 
-                uint32_t sr[128];
+                uint32_t sr[kBlockN];
                 ptx::tmem_ld128_wait(tmem_s, sr);
-                float* s = reinterpret_cast<float*>(sr);
+                float(&s)[kBlockN] = *reinterpret_cast<float(*)[kBlockN]>(sr);
 
                 const int key0 = j * kBlockN;
-                const bool need_mask = (key0 + kBlockN > p.n) || (kCausal && key0 + kBlockN - 1 > row - row_in_tile);
-                float mx;
+                const bool need_mask = (key0 + kBlockN > p.n) || (kCausal && key0 + kBlockN - 1 > tile_row0);
+                float slv = sl;
                 if (need_mask) {
-                    // Masked block (diagonal or ragged tail): scores in log2 units,
-                    // masked keys to -inf, whatever the sign of the scale.
+                    // Masked block (diagonal or ragged tail): scores to log2 units
+                    // and masked keys to -inf, whatever the sign of the scale.
                     const int limit = kCausal ? min(p.n - 1, row) : (p.n - 1);
-                    mx = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) {
-                        const float x = (key0 + c <= limit) ? s[c] * sl : -INFINITY;
-                        s[c] = x;
-                        mx = fmaxf(mx, x);
-                    }
-                } else if (sl >= 0.f) {
-                    float hi = s[0];
-#pragma unroll
-                    for (int c = 1; c < kBlockN; ++c) hi = fmaxf(hi, s[c]);
-                    mx = hi * sl;
-                } else {
-                    float lo = s[0];
-#pragma unroll
-                    for (int c = 1; c < kBlockN; ++c) lo = fminf(lo, s[c]);
-                    mx = lo * sl;
+                    for (int c = 0; c < kBlockN; ++c) s[c] = (key0 + c <= limit) ? s[c] * sl : -INFINITY;
+                    slv = 1.f;
                 }
+                const float mx = slv >= 0.f ? reduce_row<true>(s) * slv : reduce_row<false>(s) * slv;
 
                 // Online softmax update: raise the running max only when it
                 // grows by more than the threshold (the result is exact either
@@ -438,27 +521,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
 
-                float rowsum = 0.f;
-                uint32_t pk[64];
-                if (need_mask) {
-#pragma unroll
-                    for (int c = 0; c < kBlockN; c += 2) {
-                        const float p0 = ptx::ex2(s[c] - m_use);
-                        const float p1 = ptx::ex2(s[c + 1] - m_use);
-                        rowsum += p0 + p1;
-                        pk[c >> 1] = ptx::pack_bf16x2(p0, p1);
-                    }
-                } else {
-                    const float neg_m = -m_use;
-#pragma unroll
-                    for (int c = 0; c < kBlockN; c += 2) {
-                        const float p0 = ptx::ex2(fmaf(s[c], sl, neg_m));
-                        const float p1 = ptx::ex2(fmaf(s[c + 1], sl, neg_m));
-                        rowsum += p0 + p1;
-                        pk[c >> 1] = ptx::pack_bf16x2(p0, p1);
-                    }
-                }
+                uint32_t pk[kBlockN / 2];
+                float rowsum, rowsum_bf16;
+                if (need_mask)
+                    exp_block<false>(s, slv, m_use, pk, rowsum, rowsum_bf16);
+                else
+                    exp_block<true>(s, slv, m_use, pk, rowsum, rowsum_bf16);
                 l_run = l_run * alpha + rowsum;
+                lb_run = lb_run * alpha + rowsum_bf16;
                 ptx::tmem_st64(tmem_s, pk);
 
                 // Rescale this row of O_t.  S_t(j) being complete means every
@@ -481,12 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
 
             // Epilogue: O = O_acc / l, written once; lse in natural log.
-            ok = wait_bar(sync, o_full(t), o_phase);
-            ok = __all_sync(0xffffffffu, ok);
+            ok = __all_sync(0xffffffffu, wait_bar(sync, o_full(t), o_phase));
             if (!ok) break;
             o_phase ^= 1;
             ptx::tc_fence_after_sync();
-            const float inv_l = 1.f / l_run;
+            const float inv_l = 1.f / lb_run;
             const bool valid = row < p.n;
             __nv_bfloat16* orow_g = p.o + (static_cast<int64_t>(w.bh) * p.n + row) * D;
 #pragma unroll

@@ -244,5 +244,70 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// max(a, b, c) in one instruction (three-input form, sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Packed pairs of fp32 (one instruction for two lanes of work, sm_100).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// acc0 += lo(v), acc1 += hi(v) for a packed bf16 pair v (mixed-precision add).
+__device__ __forceinline__ void add_bf16x2_to_f32(float& acc0, float& acc1, uint32_t v) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(v));
+}
+
+// 2^x for two values on the FMA/ALU pipes instead of the special-function
+// unit.  Range reduction x = j + f with j = round(x), f in [-1/2, 1/2]; a cubic
+// fitted (minimax in relative error, max 7.5e-5 = 2^-13.7, see
+// fit_exp2_poly.py) gives 2^f; 2^j is added to the exponent field.  Inputs
+// below -125 are clamped there (results under 2^-125 are negligible next to
+// the row's running sum, which is at least 1).
+constexpr float kExp2C0 = 0x1.fff692p-1f;
+constexpr float kExp2C1 = 0x1.62f31ap-1f;
+constexpr float kExp2C2 = 0x1.f0de1ap-3f;
+constexpr float kExp2C3 = 0x1.c3f76p-5f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    float t0, t1, r0, r1, f0, f1, p0, p1;
+    add2(t0, t1, x0, x1, kRoundMagic, kRoundMagic);      // low mantissa bits hold round(x)
+    add2(r0, r1, t0, t1, -kRoundMagic, -kRoundMagic);    // round(x), exact
+    fma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);            // f = x - round(x)
+    fma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 }  // namespace ptx
 }  // namespace fa
