@@ -85,8 +85,13 @@ def test_f32_edge_shapes(N, d, causal):
 @pytest.mark.parametrize("scale", [-0.3, 0.0, 1.0])
 def test_scale_values(scale, dtype):
     q, k, v = W.random_qkv(1, 2, 300, 64, dtype, seed=17)
+    # scale = 1.0 at d = 64 is 8x the usual 1/sqrt(d): rows are dominated by a
+    # few keys and |O| reaches 2-4, where half a bf16 ulp of the output alone
+    # is 0.0078-0.0156; as for the Q*8 workload, the max-abs bound applies to
+    # the error beyond that rounding.
+    strict = abs(scale) <= 0.5
     for causal in (False, True):
-        check_against_oracle(q, k, v, scale, causal)
+        check_against_oracle(q, k, v, scale, causal, strict_raw=strict)
 
 
 def test_many_units_per_cta():

@@ -59,16 +59,31 @@ constexpr int kBlockM = 128;            // query rows per tile (one TMEM lane ea
 constexpr int kBlockN = 128;            // keys per KV block
 constexpr int kTilesPerUnit = 2;        // query tiles per work unit
 constexpr int kUnitRows = kBlockM * kTilesPerUnit;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
-constexpr int kThreads = 320;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxWarps = 16;       // 8 per query tile
+constexpr int kMmaWarp = 16;
+constexpr int kLoadWarp = 17;
+constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz
 constexpr int kSchedDepth = 2;              // unit ring between the producer and the other roles
 constexpr int kHeadGroup = 8;               // heads whose units are interleaved in the queue
-constexpr int kPolyPairsPer8 = 2;           // of every 8 column pairs, this many use exp2_poly2
+// Softmax tuning knobs (compile-time; -D overrides for experiments).
+#ifndef FA_POLY_PAIRS_PER8
+#define FA_POLY_PAIRS_PER8 0  // measured slower on this kernel than all-MUFU; kept as a tuning knob
+#endif
+#ifndef FA_ROWSUM_BF16
+#define FA_ROWSUM_BF16 1
+#endif
+#ifndef FA_KV_SLOTS_D128
+#define FA_KV_SLOTS_D128 4
+#endif
+#ifndef FA_PACKED_F32X2
+#define FA_PACKED_F32X2 1
+#endif
+constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;  // of every 8 column pairs, this many use exp2_poly2
+constexpr bool kRowsumBf16 = FA_ROWSUM_BF16 != 0;   // normalise O by the sum of the bf16-rounded P
+constexpr bool kPackedF32x2 = FA_PACKED_F32X2 != 0; // packed two-lane fp32 FMA/ADD
 
 template <int D>
 struct Layout {
@@ -76,15 +91,16 @@ struct Layout {
     static constexpr int kHalves = D / 64;                     // 64-column (128-byte) swizzle panels
     static constexpr int kPanelBytes = kBlockM * 128;          // one panel of a 128-row tile
     static constexpr int kTileBytes = kPanelBytes * kHalves;   // a whole 128 x D bf16 tile
-    static constexpr int kSlots = (D == 128) ? 4 : 8;          // K/V ring slots
+    static constexpr int kSlots = (D == 128) ? FA_KV_SLOTS_D128 : 8;  // K/V ring slots
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = kQOff + kTilesPerUnit * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2],
-    //           sched_full[kSchedDepth], sched_empty[kSchedDepth], drain
-    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1;
+    //           sched_full[kSchedDepth], sched_empty[kSchedDepth], drain, pair[2][4]
+    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1 + 8;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base, abort flag, unit ring
-    static constexpr int kBytes = kMiscOff + 8 + 4 * kSchedDepth;
+    static constexpr int kInvLOff = (kMiscOff + 8 + 4 * kSchedDepth + 15) & ~15;  // float[2][128]
+    static constexpr int kBytes = kInvLOff + 2 * kBlockM * 4;
     static constexpr int kSmemBytes = kBytes + 1024;           // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
     static constexpr uint32_t kTmemO = 256;
@@ -179,7 +195,12 @@ __device__ __forceinline__ void exp_block(const float (&s)[kBlockN], float slv, 
 #pragma unroll
     for (int pi = 0; pi < kBlockN / 2; ++pi) {
         float x0, x1, p0, p1;
-        ptx::fma2(x0, x1, s[2 * pi], s[2 * pi + 1], slv, slv, neg_m, neg_m);
+        if (kPackedF32x2) {
+            ptx::fma2(x0, x1, s[2 * pi], s[2 * pi + 1], slv, slv, neg_m, neg_m);
+        } else {
+            x0 = fmaf(s[2 * pi], slv, neg_m);
+            x1 = fmaf(s[2 * pi + 1], slv, neg_m);
+        }
         if (kPoly && (pi & 7) < kPolyPairsPer8) {
             ptx::exp2_poly2(p0, p1, x0, x1);
         } else {
@@ -187,28 +208,74 @@ __device__ __forceinline__ void exp_block(const float (&s)[kBlockN], float slv, 
             p1 = ptx::ex2(x1);
         }
         pk[pi] = ptx::pack_bf16x2(p0, p1);
-        ptx::add2(a[pi & 3][0], a[pi & 3][1], a[pi & 3][0], a[pi & 3][1], p0, p1);
-        ptx::add_bf16x2_to_f32(b[pi & 1][0], b[pi & 1][1], pk[pi]);
+        if (kPackedF32x2) {
+            ptx::add2(a[pi & 3][0], a[pi & 3][1], a[pi & 3][0], a[pi & 3][1], p0, p1);
+        } else {
+            a[pi & 3][0] += p0;
+            a[pi & 3][1] += p1;
+        }
+        if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[pi & 1][0], b[pi & 1][1], pk[pi]);
     }
     sum = ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
-    sum_bf16 = (b[0][0] + b[0][1]) + (b[1][0] + b[1][1]);
+    sum_bf16 = kRowsumBf16 ? (b[0][0] + b[0][1]) + (b[1][0] + b[1][1]) : sum;
 }
 
-// Row max (or min) of 128 values: eight independent chains of three-input ops.
+#ifndef FA_MAX_CHAINS
+#define FA_MAX_CHAINS 16
+#endif
+// Row max (or min) of 128 values: independent chains of three-input ops over
+// interleaved columns, then a three-way tree.
 template <bool kMax>
 __device__ __forceinline__ float reduce_row(const float (&s)[kBlockN]) {
-    float r[8];
+    constexpr int kChains = FA_MAX_CHAINS;             // 8 or 16
+    constexpr int kPer = kBlockN / kChains;             // elements per chain (16 or 8)
+    auto op3 = [](float a, float b, float c) { return kMax ? ptx::max3(a, b, c) : ptx::min3(a, b, c); };
+    auto op2 = [](float a, float b) { return kMax ? fmaxf(a, b) : fminf(a, b); };
+    float r[kChains];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float acc = s[16 * i];
+    for (int i = 0; i < kChains; ++i) {
+        float acc = op3(s[i], s[i + kChains], s[i + 2 * kChains]);
 #pragma unroll
-        for (int c = 1; c < 15; c += 2)
-            acc = kMax ? ptx::max3(acc, s[16 * i + c], s[16 * i + c + 1])
-                       : ptx::min3(acc, s[16 * i + c], s[16 * i + c + 1]);
-        r[i] = kMax ? fmaxf(acc, s[16 * i + 15]) : fminf(acc, s[16 * i + 15]);
+        for (int e = 3; e + 1 < kPer; e += 2) acc = op3(acc, s[i + e * kChains], s[i + (e + 1) * kChains]);
+        if (kPer % 2 == 0) acc = op2(acc, s[i + (kPer - 1) * kChains]);
+        r[i] = acc;
     }
-    if (kMax) return fmaxf(ptx::max3(r[0], r[1], r[2]), ptx::max3(r[3], r[4], ptx::max3(r[5], r[6], r[7])));
-    return fminf(ptx::min3(r[0], r[1], r[2]), ptx::min3(r[3], r[4], ptx::min3(r[5], r[6], r[7])));
+    // tree over the chains
+#pragma unroll
+    for (int w = kChains; w > 1;) {
+        const int n3 = w / 3, rem = w % 3;
+#pragma unroll
+        for (int i = 0; i < n3; ++i) r[i] = op3(r[3 * i], r[3 * i + 1], r[3 * i + 2]);
+        if (rem == 1) r[n3] = r[3 * n3];
+        if (rem == 2) r[n3] = op2(r[3 * n3], r[3 * n3 + 1]);
+        w = n3 + (rem ? 1 : 0);
+    }
+    return r[0];
+}
+
+// Max (or min) of each of this thread's two rows (64 values in the .16x256b
+// register order: 4k + {0,1} first row, 4k + {2,3} second row) completed
+// across the quad that shares the rows.
+template <bool kMax>
+__device__ __forceinline__ void quad_row_extreme(const float (&s)[64], float (&out)[2]) {
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : fminf(a, b); };
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        float c0 = s[2 * r], c1 = s[2 * r + 1], c2 = s[4 + 2 * r], c3 = s[5 + 2 * r];
+#pragma unroll
+        for (int k = 2; k < 16; k += 2) {
+            c0 = op(c0, s[4 * k + 2 * r]);
+            c1 = op(c1, s[4 * k + 2 * r + 1]);
+            c2 = op(c2, s[4 * k + 4 + 2 * r]);
+            c3 = op(c3, s[4 * k + 5 + 2 * r]);
+        }
+        out[r] = op(op(c0, c1), op(c2, c3));
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        out[r] = op(out[r], __shfl_xor_sync(0xffffffffu, out[r], 1));
+        out[r] = op(out[r], __shfl_xor_sync(0xffffffffu, out[r], 2));
+    }
 }
 
 template <int D, bool kCausal>
@@ -237,6 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto sched_full = [&](int i) { return bar0 + 8u * (10 + 2 * L::kSlots + i); };
     auto sched_empty = [&](int i) { return bar0 + 8u * (10 + 2 * L::kSlots + kSchedDepth + i); };
     const uint32_t drain = bar0 + 8u * (10 + 2 * L::kSlots + 2 * kSchedDepth);
+    // the two softmax warps of tile t that share TMEM lane quarter q meet here in the epilogue
+    auto pair_bar = [&](int t, int q) { return bar0 + 8u * (11 + 2 * L::kSlots + 2 * kSchedDepth + 4 * t + q); };
 
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -248,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(q_full(t), 1);
             ptx::mbar_init(q_empty(t), 1);
             ptx::mbar_init(s_full(t), 1);
-            ptx::mbar_init(p_full(t), kBlockM);
+            ptx::mbar_init(p_full(t), 32 * (kSoftmaxWarps / 2));
+            for (int q = 0; q < 4; ++q) ptx::mbar_init(pair_bar(t, q), 64);
             ptx::mbar_init(o_full(t), 1);
         }
         for (int s = 0; s < L::kSlots; ++s) {
@@ -279,63 +349,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t keep = ptx::policy_evict_last();   // K/V: re-read by the head's other units
-            const uint64_t once = ptx::policy_evict_first();  // Q: read once
-            int slot = 0;
-            uint32_t phase = 0;
-            // last issued phase per slot (+1), for draining
-            uint32_t slot_issued[L::kSlots];
-            uint32_t q_issued[2] = {0, 0};
-            for (int s = 0; s < L::kSlots; ++s) slot_issued[s] = 0;
-            bool ok = true;
-            for (uint32_t it = 0; ok; ++it) {
-                // take the next unit from the queue and publish it to the CTA
-                const int rs = it % kSchedDepth;
-                ok = wait_bar(sync, sched_empty(rs), ((it / kSchedDepth) & 1) ^ 1);
-                if (!ok) break;
-                int u = static_cast<int>(atomicAdd(p.sched, 1u));
+        // The whole warp runs the loop (warp-uniform addresses and waits);
+        // one elected lane issues the copies.
+        const bool leader = ptx::elect_one();
+        const uint64_t keep = ptx::policy_evict_last();   // K/V: re-read by the head's other units
+        const uint64_t once = ptx::policy_evict_first();  // Q: read once
+        int slot = 0;
+        uint32_t phase = 0, nloads = 0;
+        uint32_t q_issued[2] = {0, 0};  // last issued phase of each Q slot (+1), for draining
+        bool ok = true;
+        for (uint32_t it = 0; ok; ++it) {
+            // take the next unit from the queue and publish it to the CTA
+            const int rs = it % kSchedDepth;
+            ok = __all_sync(0xffffffffu, wait_bar(sync, sched_empty(rs), ((it / kSchedDepth) & 1) ^ 1));
+            if (!ok) break;
+            int u = 0;
+            if (leader) {
+                u = static_cast<int>(atomicAdd(p.sched, 1u));
                 if (u >= p.num_units) u = -1;
                 unit_ring[rs] = u;
                 ptx::mbar_arrive(sched_full(rs));
-                if (u < 0) break;
+            }
+            u = __shfl_sync(0xffffffffu, u, __ffs(__ballot_sync(0xffffffffu, leader)) - 1);
+            if (u < 0) break;
 
-                const Unit w = decode_unit(u, p, kCausal);
-                const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
-                for (int t = 0; t < 2 && ok; ++t) {
-                    ok = wait_bar(sync, q_empty(t), (it & 1) ^ 1);
-                    if (!ok) break;
-                    const uint32_t dst = base + L::kQOff + t * L::kTileBytes;
+            const Unit w = decode_unit(u, p, kCausal);
+            const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!ok) break;
+                ok = __all_sync(0xffffffffu, wait_bar(sync, q_empty(t), (it & 1) ^ 1));
+                if (!ok) break;
+                const uint32_t dst = base + L::kQOff + t * L::kTileBytes;
+                q_issued[t] = (it & 1) + 1;
+                if (leader) {
                     ptx::mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
-                    q_issued[t] = (it & 1) + 1;
                     for (int h = 0; h < L::kHalves; ++h)
                         ptx::tma_load_3d(dst + h * L::kPanelBytes, &tm_q, q_full(t), h * 64,
                                          w.qb * kUnitRows + t * kBlockM, w.bh, once);
                 }
-                for (int j = 0; j < n1 && ok; ++j) {
-                    for (int kv = 0; kv < 2 && ok; ++kv) {
-                        ok = wait_bar(sync, kv_empty(slot), phase ^ 1);
-                        if (!ok) break;
-                        const uint32_t dst = base + L::kRingOff + slot * L::kTileBytes;
+            }
+            for (int j = 0; j < n1 && ok; ++j) {
+                for (int kv = 0; kv < 2 && ok; ++kv) {
+                    ok = __all_sync(0xffffffffu, wait_bar(sync, kv_empty(slot), phase ^ 1));
+                    if (!ok) break;
+                    const uint32_t dst = base + L::kRingOff + slot * L::kTileBytes;
+                    if (leader) {
                         ptx::mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
-                        slot_issued[slot] = phase + 1;
                         const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
                         for (int h = 0; h < L::kHalves; ++h)
                             ptx::tma_load_3d(dst + h * L::kPanelBytes, tm, kv_full(slot), h * 64,
                                              j * kBlockN, w.bh, keep);
-                        if (++slot == L::kSlots) {
-                            slot = 0;
-                            phase ^= 1;
-                        }
+                    }
+                    ++nloads;
+                    if (++slot == L::kSlots) {
+                        slot = 0;
+                        phase ^= 1;
                     }
                 }
             }
-            // Drain: every issued copy must land before shared memory is released.
-            for (int s = 0; s < L::kSlots; ++s)
-                if (slot_issued[s]) drain_bar(sync, kv_full(s), slot_issued[s] - 1);
-            for (int t = 0; t < 2; ++t)
-                if (q_issued[t]) drain_bar(sync, q_full(t), q_issued[t] - 1);
-            // The last CTA to finish returns the queue to zero for the next launch.
+        }
+        // Drain: every issued copy must land before shared memory is released.
+        // Load i went to slot i % S with phase (i / S) & 1.
+        for (uint32_t s = 0; s < static_cast<uint32_t>(L::kSlots) && s < nloads; ++s) {
+            const uint32_t last = s + L::kSlots * ((nloads - 1 - s) / L::kSlots);
+            drain_bar(sync, kv_full(s), (last / L::kSlots) & 1);
+        }
+        for (int t = 0; t < 2; ++t)
+            if (q_issued[t]) drain_bar(sync, q_full(t), q_issued[t] - 1);
+        // The last CTA to finish returns the queue to zero for the next launch.
+        if (leader) {
             __threadfence();
             if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
                 atomicExch(p.sched, 0u);
@@ -345,126 +428,149 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = ptx::make_idesc_bf16(kBlockM, kBlockN, false);
-            constexpr uint32_t idesc_o = ptx::make_idesc_bf16(kBlockM, D, true);
-            int slot = 0;
-            uint32_t phase = 0;
-            uint32_t p_phase[2] = {0, 0};
-            bool ok = true;
+        // The whole warp runs the loop and builds the descriptors (so they are
+        // warp-uniform); one elected lane issues every MMA and commit.
+        const bool leader = ptx::elect_one();
+        constexpr uint32_t idesc_s = ptx::make_idesc_bf16(kBlockM, kBlockN, false);
+        constexpr uint32_t idesc_o = ptx::make_idesc_bf16(kBlockM, D, true);
+        // base descriptors; operand offsets are added to the start-address field
+        const uint64_t desc_q0 = ptx::make_smem_desc(base + L::kQOff, 16, 1024);
+        const uint64_t desc_k0 = ptx::make_smem_desc(base + L::kRingOff, 16, 1024);
+        const uint64_t desc_v0 = ptx::make_smem_desc(base + L::kRingOff, L::kPanelBytes, 1024);
+        int slot = 0;
+        uint32_t phase = 0;
+        uint32_t p_phase[2] = {0, 0};
+        bool ok = true;
 
-            // S_t = Q_t K^T over the head dim: D/16 MMAs of K = 16.
-            auto issue_s = [&](int t, int kslot) {
-                const uint32_t q_base = base + L::kQOff + t * L::kTileBytes;
-                const uint32_t k_base = base + L::kRingOff + kslot * L::kTileBytes;
+        // S_t = Q_t K^T over the head dim: D/16 MMAs of K = 16.
+        auto issue_s = [&](int t, int kslot) {
+            const uint64_t qd = desc_q0 + ((t * L::kTileBytes) >> 4);
+            const uint64_t kd = desc_k0 + ((kslot * L::kTileBytes) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * L::kPanelBytes + (ks & 3) * 32;
-                    const uint64_t a = ptx::make_smem_desc(q_base + off, 16, 1024);
-                    const uint64_t b = ptx::make_smem_desc(k_base + off, 16, 1024);
-                    ptx::mma_ss(tmem + L::kTmemS + t * kBlockN, a, b, idesc_s, ks > 0);
-                }
-            };
-            // O_t (+)= P_t V: 128/16 MMAs; P from TMEM (8 columns per 16 keys),
-            // V from shared memory as an MN-major operand (d contiguous).
-            auto issue_pv = [&](int t, int vslot, bool accumulate) {
-                const uint32_t v_base = base + L::kRingOff + vslot * L::kTileBytes;
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t off = ((ks >> 2) * L::kPanelBytes + (ks & 3) * 32) >> 4;
+                if (leader) ptx::mma_ss(tmem + L::kTmemS + t * kBlockN, qd + off, kd + off, idesc_s, ks > 0);
+            }
+        };
+        // O_t (+)= P_t V: 128/16 MMAs; P from TMEM (8 columns per 16 keys),
+        // V from shared memory as an MN-major operand (d contiguous).
+        auto issue_pv = [&](int t, int vslot, bool accumulate) {
+            const uint64_t vd = desc_v0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < kBlockN / 16; ++ks) {
-                    const uint64_t b = ptx::make_smem_desc(v_base + ks * 16 * 128, L::kPanelBytes, 1024);
-                    ptx::mma_ts(tmem + L::kTmemO + t * D, tmem + L::kTmemS + t * kBlockN + ks * 8, b,
-                                idesc_o, (accumulate || ks > 0) ? 1u : 0u);
-                }
-            };
-            auto next_slot = [&](int& s, uint32_t& ph) {
-                s = slot;
-                ph = phase;
-                if (++slot == L::kSlots) {
-                    slot = 0;
-                    phase ^= 1;
-                }
-            };
+            for (int ks = 0; ks < kBlockN / 16; ++ks) {
+                if (leader)
+                    ptx::mma_ts(tmem + L::kTmemO + t * D, tmem + L::kTmemS + t * kBlockN + ks * 8,
+                                vd + ((ks * 16 * 128) >> 4), idesc_o, (accumulate || ks > 0) ? 1u : 0u);
+            }
+        };
+        auto commit = [&](uint32_t bar) {
+            if (leader) ptx::mma_commit(bar);
+        };
+        auto next_slot = [&](int& s, uint32_t& ph) {
+            s = slot;
+            ph = phase;
+            if (++slot == L::kSlots) {
+                slot = 0;
+                phase ^= 1;
+            }
+        };
+        auto wait_all = [&](uint32_t bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, wait_bar(sync, bar, parity));
+        };
 
-            for (uint32_t it = 0; ok; ++it) {
-                const int rs = it % kSchedDepth;
-                ok = wait_bar(sync, sched_full(rs), (it / kSchedDepth) & 1);
-                if (!ok) break;
-                const int u = unit_ring[rs];
-                ptx::mbar_arrive(sched_empty(rs));
-                if (u < 0) break;
+        for (uint32_t it = 0; ok; ++it) {
+            const int rs = it % kSchedDepth;
+            ok = wait_all(sched_full(rs), (it / kSchedDepth) & 1);
+            if (!ok) break;
+            const int u = unit_ring[rs];
+            __syncwarp();
+            if (leader) ptx::mbar_arrive(sched_empty(rs));
+            if (u < 0) break;
 
-                const Unit w = decode_unit(u, p, kCausal);
-                const int n0 = num_kv_blocks(p, w.qb, 0, kCausal);
-                const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
-                ok = wait_bar(sync, q_full(0), it & 1) && wait_bar(sync, q_full(1), it & 1);
-                if (!ok) break;
-                int sk, sv;
-                uint32_t pk, pv;
-                next_slot(sk, pk);
-                ok = wait_bar(sync, kv_full(sk), pk);
-                if (!ok) break;
-                ptx::tc_fence_after_sync();
-                issue_s(0, sk);
-                ptx::mma_commit(s_full(0));
-                if (n0 == 1) ptx::mma_commit(q_empty(0));
-                issue_s(1, sk);
-                ptx::mma_commit(s_full(1));
-                if (n1 == 1) ptx::mma_commit(q_empty(1));
-                ptx::mma_commit(kv_empty(sk));
+            const Unit w = decode_unit(u, p, kCausal);
+            const int n0 = num_kv_blocks(p, w.qb, 0, kCausal);
+            const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
+            ok = wait_all(q_full(0), it & 1) && wait_all(q_full(1), it & 1);
+            if (!ok) break;
+            int sk, sv;
+            uint32_t pk, pv;
+            next_slot(sk, pk);
+            ok = wait_all(kv_full(sk), pk);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            issue_s(0, sk);
+            commit(s_full(0));
+            if (n0 == 1) commit(q_empty(0));
+            issue_s(1, sk);
+            commit(s_full(1));
+            if (n1 == 1) commit(q_empty(1));
+            commit(kv_empty(sk));
 
-                for (int j = 0; j < n1 && ok; ++j) {
-                    next_slot(sv, pv);
-                    ok = wait_bar(sync, kv_full(sv), pv);
+            for (int j = 0; j < n1 && ok; ++j) {
+                next_slot(sv, pv);
+                ok = wait_all(kv_full(sv), pv);
+                if (!ok) break;
+                if (j < n0) {
+                    ok = wait_all(p_full(0), p_phase[0]);
                     if (!ok) break;
-                    if (j < n0) {
-                        ok = wait_bar(sync, p_full(0), p_phase[0]);
-                        if (!ok) break;
-                        p_phase[0] ^= 1;
-                        ptx::tc_fence_after_sync();
-                        issue_pv(0, sv, j > 0);
-                        if (j == n0 - 1) ptx::mma_commit(o_full(0));
-                    }
-                    const bool more = j + 1 < n1;
-                    if (more) {
-                        next_slot(sk, pk);
-                        ok = wait_bar(sync, kv_full(sk), pk);
-                        if (!ok) break;
-                        ptx::tc_fence_after_sync();
-                    }
-                    if (j + 1 < n0) {
-                        issue_s(0, sk);
-                        ptx::mma_commit(s_full(0));
-                        if (j + 1 == n0 - 1) ptx::mma_commit(q_empty(0));
-                    }
-                    ok = wait_bar(sync, p_full(1), p_phase[1]);
-                    if (!ok) break;
-                    p_phase[1] ^= 1;
+                    p_phase[0] ^= 1;
                     ptx::tc_fence_after_sync();
-                    issue_pv(1, sv, j > 0);
-                    if (j == n1 - 1) ptx::mma_commit(o_full(1));
-                    ptx::mma_commit(kv_empty(sv));
-                    if (more) {
-                        issue_s(1, sk);
-                        ptx::mma_commit(s_full(1));
-                        if (j + 1 == n1 - 1) ptx::mma_commit(q_empty(1));
-                        ptx::mma_commit(kv_empty(sk));
-                    }
+                    issue_pv(0, sv, j > 0);
+                    if (j == n0 - 1) commit(o_full(0));
+                }
+                const bool more = j + 1 < n1;
+                if (more) {
+                    next_slot(sk, pk);
+                    ok = wait_all(kv_full(sk), pk);
+                    if (!ok) break;
+                    ptx::tc_fence_after_sync();
+                }
+                if (j + 1 < n0) {
+                    issue_s(0, sk);
+                    commit(s_full(0));
+                    if (j + 1 == n0 - 1) commit(q_empty(0));
+                }
+                ok = wait_all(p_full(1), p_phase[1]);
+                if (!ok) break;
+                p_phase[1] ^= 1;
+                ptx::tc_fence_after_sync();
+                issue_pv(1, sv, j > 0);
+                if (j == n1 - 1) commit(o_full(1));
+                commit(kv_empty(sv));
+                if (more) {
+                    issue_s(1, sk);
+                    commit(s_full(1));
+                    if (j + 1 == n1 - 1) commit(q_empty(1));
+                    commit(kv_empty(sk));
                 }
             }
-            // Drain: all issued MMAs complete before TMEM is released.
-            ptx::mma_commit(drain);
-            drain_bar(sync, drain, 0);
         }
+        // Drain: all issued MMAs complete before TMEM is released.
+        commit(drain);
+        drain_bar(sync, drain, 0);
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        const int t = warp >> 2;                         // query tile of this warpgroup
-        const int row_in_tile = (warp & 3) * 32 + lane;  // TMEM lane == tile row
-        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        // ------------------------------------------------------------ softmax warps
+        // Warps 0-7 serve query tile 0 and warps 8-15 tile 1.  The two warps
+        // of a tile that share TMEM lane quarter q (= warp % 4) split its 32
+        // rows: half h covers rows 32q + 16h .. +15, read with the 16-lane
+        // TMEM shapes.  A quad of threads (lane / 4) owns two rows, r0 and
+        // r0 + 8, and in every 8-column chunk k the column pair
+        // 8k + 2(lane % 4) + {0, 1}; row reductions finish with two shuffles
+        // inside the quad.
+        const int t = warp >> 3;
+        const int q = warp & 3;
+        const int h = (warp >> 2) & 1;
+        const int qc = lane & 3;                          // column pair within each chunk
+        const int rr0 = 32 * q + 16 * h + (lane >> 2);    // row-in-tile of r0 (r1 = rr0 + 8)
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q + 16 * h) << 16;
         const uint32_t tmem_s = tmem + lane_addr + L::kTmemS + t * kBlockN;
         const uint32_t tmem_o = tmem + lane_addr + L::kTmemO + t * D;
+        // one-row-per-thread view of the same lane quarter, for the epilogue
+        const uint32_t tmem_o_rows = tmem + (static_cast<uint32_t>(32 * q) << 16) + L::kTmemO + t * D;
+        float* inv_l_sm = reinterpret_cast<float*>(smem + L::kInvLOff) + t * kBlockM;
         const float sl = p.scale_log2;
-        uint32_t s_phase = 0, o_phase = 0;
+        uint32_t s_phase = 0, o_phase = 0, pair_phase = 0;
         bool ok = true;
 
         for (uint32_t it = 0; ok; ++it) {
@@ -479,10 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Unit w = decode_unit(u, p, kCausal);
             const int nt = num_kv_blocks(p, w.qb, t, kCausal);
             const int tile_row0 = w.qb * kUnitRows + t * kBlockM;
-            const int row = tile_row0 + row_in_tile;
-            float m_run = -INFINITY;  // running max, log2 units (scale folded in)
-            float l_run = 0.f;        // running sum of 2^(x - m_run), fp32
-            float lb_run = 0.f;       // the same sum over the bf16-rounded values
+            const int row0 = tile_row0 + rr0;                 // global rows of r0 and r1
+            const int row1 = row0 + 8;
+            float m_run[2] = {-INFINITY, -INFINITY};  // running max per row, log2 units
+            float l_run[2] = {0.f, 0.f};              // partial (this thread's columns) fp32 sums
+            float lb_run[2] = {0.f, 0.f};             // the same over the bf16-rounded values
 
             for (int j = 0; j < nt; ++j) {
                 ok = __all_sync(0xffffffffu, wait_bar(sync, s_full(t), s_phase));
@@ -490,9 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_phase ^= 1;
                 ptx::tc_fence_after_sync();
 
-                uint32_t sr[kBlockN];
-                ptx::tmem_ld128_wait(tmem_s, sr);
-                float(&s)[kBlockN] = *reinterpret_cast<float(*)[kBlockN]>(sr);
+                uint32_t sr[64];
+                ptx::tmem_ld16x256b_x16_wait(tmem_s, sr);
+                float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
 
                 const int key0 = j * kBlockN;
                 const bool need_mask = (key0 + kBlockN > p.n) || (kCausal && key0 + kBlockN - 1 > tile_row0);
@@ -500,48 +607,88 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (need_mask) {
                     // Masked block (diagonal or ragged tail): scores to log2 units
                     // and masked keys to -inf, whatever the sign of the scale.
-                    const int limit = kCausal ? min(p.n - 1, row) : (p.n - 1);
+                    const int lim0 = kCausal ? min(p.n - 1, row0) : (p.n - 1);
+                    const int lim1 = kCausal ? min(p.n - 1, row1) : (p.n - 1);
 #pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) s[c] = (key0 + c <= limit) ? s[c] * sl : -INFINITY;
+                    for (int k = 0; k < 16; ++k)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int key = key0 + 8 * k + 2 * qc + (i & 1);
+                            const int lim = (i < 2) ? lim0 : lim1;
+                            s[4 * k + i] = (key <= lim) ? s[4 * k + i] * sl : -INFINITY;
+                        }
                     slv = 1.f;
                 }
-                const float mx = slv >= 0.f ? reduce_row<true>(s) * slv : reduce_row<false>(s) * slv;
-
-                // Online softmax update: raise the running max only when it
-                // grows by more than the threshold (the result is exact either
-                // way: O and l always share the same m).
-                float alpha = 1.f;
-                bool rescale_o = false;
-                if (j == 0) {
-                    m_run = mx;
-                } else if (mx > m_run + kRescaleThreshold) {
-                    alpha = ptx::ex2(m_run - mx);
-                    m_run = mx;
-                    rescale_o = true;
-                }
-                const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-
-                uint32_t pk[kBlockN / 2];
-                float rowsum, rowsum_bf16;
-                if (need_mask)
-                    exp_block<false>(s, slv, m_use, pk, rowsum, rowsum_bf16);
+                // row max (or min for a negative scale) over this thread's 32
+                // values per row, then across the quad
+                float mx[2];
+                if (slv >= 0.f)
+                    quad_row_extreme<true>(s, mx);
                 else
-                    exp_block<true>(s, slv, m_use, pk, rowsum, rowsum_bf16);
-                l_run = l_run * alpha + rowsum;
-                lb_run = lb_run * alpha + rowsum_bf16;
-                ptx::tmem_st64(tmem_s, pk);
+                    quad_row_extreme<false>(s, mx);
+                mx[0] *= slv;
+                mx[1] *= slv;
 
-                // Rescale this row of O_t.  S_t(j) being complete means every
+                // Online softmax update per row: raise the running max only
+                // when it grows by more than the threshold (the result is exact
+                // either way: O and l always share the same m).
+                float alpha[2] = {1.f, 1.f}, neg_m[2];
+                bool rescale_o = false;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    if (j == 0) {
+                        m_run[r] = mx[r];
+                    } else if (mx[r] > m_run[r] + kRescaleThreshold) {
+                        alpha[r] = ptx::ex2(m_run[r] - mx[r]);
+                        m_run[r] = mx[r];
+                        rescale_o = true;
+                    }
+                    neg_m[r] = (m_run[r] == -INFINITY) ? 0.f : -m_run[r];
+                }
+
+                // p = 2^(s * slv - m): packed bf16 pairs, pk[2k] for r0 and
+                // pk[2k + 1] for r1 in chunk k (the .16x128b store order), and
+                // both row sums.  Unmasked blocks send part of the pairs through
+                // the polynomial on the FMA pipe.
+                uint32_t pk[32];
+                float a[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                float b[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        float x0, x1, p0, p1;
+                        ptx::fma2(x0, x1, s[4 * k + 2 * r], s[4 * k + 2 * r + 1], slv, slv, neg_m[r], neg_m[r]);
+                        if (!need_mask && ((2 * k + r) & 7) < kPolyPairsPer8) {
+                            ptx::exp2_poly2(p0, p1, x0, x1);
+                        } else {
+                            p0 = ptx::ex2(x0);
+                            p1 = ptx::ex2(x1);
+                        }
+                        const uint32_t v = ptx::pack_bf16x2(p0, p1);
+                        pk[2 * k + r] = v;
+                        ptx::add2(a[r][0], a[r][1], a[r][0], a[r][1], p0, p1);
+                        if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[r][0], b[r][1], v);
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    l_run[r] = l_run[r] * alpha[r] + (a[r][0] + a[r][1]);
+                    lb_run[r] = lb_run[r] * alpha[r] + (kRowsumBf16 ? (b[r][0] + b[r][1]) : (a[r][0] + a[r][1]));
+                }
+                ptx::tmem_st16x128b_x16(tmem_s, pk);
+
+                // Rescale these rows of O_t.  S_t(j) being complete means every
                 // earlier MMA (PV_t(j-1) included) is complete, so O_t is stable.
                 if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t orow[32];
-                        ptx::tmem_ld32_wait(tmem_o + c0, orow);
+                        uint32_t ov[16];
+                        ptx::tmem_ld16x256b_x4_wait(tmem_o + c0, ov);
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha);
-                        ptx::tmem_st32(tmem_o + c0, orow);
+                        for (int i = 0; i < 16; ++i)
+                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha[(i >> 1) & 1]);
+                        ptx::tmem_st16x256b_x4(tmem_o + c0, ov);
                     }
                 }
                 ptx::tmem_st_wait();
@@ -550,18 +697,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
 
-            // Epilogue: O = O_acc / l, written once; lse in natural log.
+            // Epilogue.  Row sums are complete once added across the quad.
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+                l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+                lb_run[r] += __shfl_xor_sync(0xffffffffu, lb_run[r], 1);
+                lb_run[r] += __shfl_xor_sync(0xffffffffu, lb_run[r], 2);
+            }
             ok = __all_sync(0xffffffffu, wait_bar(sync, o_full(t), o_phase));
             if (!ok) break;
             o_phase ^= 1;
             ptx::tc_fence_after_sync();
-            const float inv_l = 1.f / lb_run;
+            if (qc == 0) {
+                inv_l_sm[rr0] = 1.f / lb_run[0];
+                inv_l_sm[rr0 + 8] = 1.f / lb_run[1];
+                // lse in natural log, written once per row
+                const float mu0 = (m_run[0] == -INFINITY) ? 0.f : m_run[0];
+                const float mu1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
+                if (row0 < p.n) p.lse[static_cast<int64_t>(w.bh) * p.n + row0] = (mu0 + log2f(l_run[0])) * 0.69314718055994531f;
+                if (row1 < p.n) p.lse[static_cast<int64_t>(w.bh) * p.n + row1] = (mu1 + log2f(l_run[1])) * 0.69314718055994531f;
+            }
+            // both warps of the lane quarter have published their rows' 1/l
+            ptx::mbar_arrive(pair_bar(t, q));
+            ok = __all_sync(0xffffffffu, wait_bar(sync, pair_bar(t, q), pair_phase));
+            if (!ok) break;
+            pair_phase ^= 1;
+            // O = O_acc / l, written once: this warp stores columns
+            // [D/2 h, D/2 (h+1)) of the quarter's 32 rows, one row per thread.
+            const int row = tile_row0 + 32 * q + lane;
+            const float inv_l = inv_l_sm[32 * q + lane];
             const bool valid = row < p.n;
-            __nv_bfloat16* orow_g = p.o + (static_cast<int64_t>(w.bh) * p.n + row) * D;
+            __nv_bfloat16* orow_g = p.o + (static_cast<int64_t>(w.bh) * p.n + row) * D + (D / 2) * h;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
                 uint32_t acc[32];
-                ptx::tmem_ld32_wait(tmem_o + c0, acc);
+                ptx::tmem_ld32_wait(tmem_o_rows + (D / 2) * h + c0, acc);
                 uint32_t packed[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2)
@@ -574,10 +745,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
                                             packed[4 * v + 3]);
                 }
-            }
-            if (valid) {
-                const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                p.lse[static_cast<int64_t>(w.bh) * p.n + row] = (m_use + log2f(l_run)) * 0.69314718055994531f;
             }
             ptx::tc_fence_before_sync();
         }
