@@ -83,6 +83,37 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            float scale, int causal, int dtype, void* stream);
 
 /*
+ * fa_fwd_noalloc -- fa_fwd for callers that must not allocate device memory.
+ * The pages have no counterpart: this is a deployment variant of the same
+ * call, not part of the method.
+ *
+ * fa_fwd allocates a small device workspace (status word and work-queue
+ * counters) with cudaMalloc on its first call on each device.  Callers that
+ * cannot allow a library to allocate -- a serving process that has already
+ * reserved all GPU memory for its own pool, code running inside an
+ * allocator's hooks, strict per-library memory budgets -- use this entry
+ * point instead: same arguments, layouts, results and errors as fa_fwd, but
+ * the scratch lives in a fixed 256-byte device array that the library
+ * carries (every GPU that loads the library holds it until the process
+ * exits), and no allocating routine is called.
+ *
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - Each call clears the array's status and queue words on `stream` before
+ *     its kernel runs.  All calls share the one array: calls whose kernels can
+ *     overlap on the GPU (different streams, several host threads) race on it
+ *     and give wrong results; issue them in order on one stream.
+ *   - A call that would need more scratch than the array holds is rejected
+ *     with FA_ERR_UNSUPPORTED (the current kernels need 24 bytes).
+ *   - A device-side timeout of a call made here is recorded only in the array,
+ *     not reported by fa_check_device_status.
+ */
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int64_t B, int64_t H, int64_t N, int64_t d,
+                   float scale, int causal, int dtype, void* stream);
+
+/*
  * fa_check_device_status -- synchronise `stream`, then read and clear the
  * library's device status word for the current device.  Returns FA_OK,
  * FA_ERR_DEVICE_TIMEOUT when a kernel launched by this library gave up on a

@@ -271,3 +271,161 @@ int fa_check_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_fwd_noalloc: the same forward for callers that must not allocate device
+// memory.  fa_fwd allocates a small workspace (device status word and
+// work-queue counters) with cudaMalloc on its first call on each device; some
+// callers cannot let a library do that -- a serving process that has already
+// reserved the whole GPU memory for its own pool, code that runs inside an
+// allocator's hooks, or deployments with strict per-library memory budgets.
+// This entry point keeps that scratch in a fixed, file-scope device array
+// instead and calls no allocating routine.
+namespace {
+
+// 256 bytes of scratch, loaded with the library on every GPU it runs on and
+// kept until the process exits.  Word 0: device status (a kernel that gave up
+// on a bounded wait sets it); words 4 and 5: the persistent kernel's work
+// queue (next unit, CTAs finished).  The rest is unused headroom.
+constexpr int kNoAllocScratchWords = 64;
+constexpr int kNoAllocStatusWord = 0;
+constexpr int kNoAllocQueueWord = 4;
+constexpr int kNoAllocWordsUsed = 6;
+static __device__ __align__(256) unsigned g_noalloc_scratch[kNoAllocScratchWords];
+static_assert(kNoAllocWordsUsed <= kNoAllocScratchWords, "no-alloc scratch too small");
+
+struct NoAllocDevice {
+    bool ready = false;
+    unsigned* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+    int sm_count = 0;
+    int cc_major = 0;
+    bool smem_raised[4] = {false, false, false, false};
+};
+NoAllocDevice g_noalloc_dev[kMaxDevices];
+
+// First call on a device (with that device current): look up the scratch
+// array's device address and the launch attributes.  Nothing is allocated.
+int noalloc_setup(NoAllocDevice** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lock(g_mu);
+    NoAllocDevice& s = g_noalloc_dev[dev];
+    if (!s.ready) {
+        if ((e = cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+        if ((e = cudaDeviceGetAttribute(&s.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute(compute capability)");
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void* fn = nullptr;
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+                return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        void* ptr = nullptr;
+        if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        s.scratch = static_cast<unsigned*>(ptr);
+        s.ready = true;
+    }
+    *out = &s;
+    return FA_OK;
+}
+
+template <int D, bool kCausal>
+int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* k, const void* v, void* o,
+                        float* lse, int64_t bh, int64_t n, float scale, cudaStream_t stream) {
+    using L = fa::tc::Layout<D>;
+    auto kernel = fa::tc::fa_fwd_bf16_kernel<D, kCausal>;
+    if (!st->smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->smem_raised[slot] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+    // The array keeps the previous call's contents: the status word and the
+    // queue counters must start at zero, so clear them in stream order.
+    cudaError_t e = cudaMemsetAsync(st->scratch, 0, kNoAllocWordsUsed * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc scratch)");
+
+    fa::tc::Params p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.status = reinterpret_cast<int*>(st->scratch + kNoAllocStatusWord);
+    p.sched = st->scratch + kNoAllocQueueWord;
+    p.bh = static_cast<int>(bh);
+    p.n = static_cast<int>(n);
+    p.num_qblocks = static_cast<int>((n + fa::tc::kUnitRows - 1) / fa::tc::kUnitRows);
+    p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
+    p.num_units = p.bh * p.num_qblocks;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
+    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the bf16 attention kernel (no-alloc)");
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                              int64_t H, int64_t N, int64_t d, float scale, int causal, int dtype,
+                              void* stream) {
+    g_last_error.clear();
+    // ---- the same argument checks as fa_fwd, before any CUDA call
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    const int64_t bh = B * H;
+    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
+    const int64_t units = bh * ((N + 255) / 256);
+    if (units > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
+    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
+    if (bh > (int64_t{1} << 62) / (N * d * elem)) return fail(FA_ERR_INVALID_ARGUMENT, "tensor size overflows");
+    const size_t tensor_bytes = static_cast<size_t>(bh * N * d * elem);
+    const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
+    auto misaligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) != 0; };
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16))
+        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+    if (misaligned(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
+        overlaps(o, tensor_bytes, v, tensor_bytes) || overlaps(o, tensor_bytes, lse, lse_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
+    if (overlaps(lse, lse_bytes, q, tensor_bytes) || overlaps(lse, lse_bytes, k, tensor_bytes) ||
+        overlaps(lse, lse_bytes, v, tensor_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
+    // the scratch this call needs must fit the fixed array
+    if (static_cast<size_t>(kNoAllocWordsUsed) * sizeof(unsigned) > sizeof(g_noalloc_scratch))
+        return fail(FA_ERR_UNSUPPORTED, "call needs more scratch than the 256-byte no-alloc array holds");
+
+    // ---- set-up on the first call per device (no allocation) and dispatch
+    NoAllocDevice* st = nullptr;
+    int rc = noalloc_setup(&st);
+    if (rc != FA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool c = causal != 0;
+    if (dtype == FA_DTYPE_BF16) {
+        if (st->cc_major != 10)
+            return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
+        if (d == 128) return c ? launch_bf16_noalloc<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
+                               : launch_bf16_noalloc<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
+        return c ? launch_bf16_noalloc<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
+                 : launch_bf16_noalloc<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
+    }
+    // the fp32 kernel uses no scratch at all
+    if (d == 128) return c ? launch_f32<128, true>(q, k, v, o, lse, bh, N, scale, s)
+                           : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
+    return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
+             : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+}
