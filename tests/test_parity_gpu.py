@@ -196,3 +196,19 @@ def test_two_streams_interleaved():
     fa.check_device_status()
     for o, lse in outs:
         assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_growing_scores_take_the_slow_path(d, causal):
+    # Scores rise by about 58 log2-units along the sequence (~7 per 128-key
+    # block), so the running max of every row falls far enough behind to make
+    # the kernel redo blocks against their exact max several times per row.
+    N = 1024
+    g = torch.Generator().manual_seed(61)
+    q = torch.ones(1, 2, N, d)
+    ramp = torch.linspace(0, 40.0 * 8 / d, N).view(1, 1, N, 1)
+    k = (ramp + 0.05 * torch.randn(1, 2, N, d, generator=g)).expand(1, 2, N, d)
+    v = torch.randn(1, 2, N, d, generator=g)
+    q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
+    check_against_oracle(q, k, v, 1.0 / 8.0, causal, strict_raw=False)

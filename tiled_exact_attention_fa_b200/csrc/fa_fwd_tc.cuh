@@ -64,7 +64,7 @@ constexpr int kMmaWarp = 16;
 constexpr int kLoadWarp = 17;
 constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
+constexpr float kStaleMaxBound = 1048576.0f;  // 2^20: largest p accepted against a stale running max
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz
 constexpr int kSchedDepth = 2;              // unit ring between the producer and the other roles
 constexpr int kHeadGroup = 8;               // heads whose units are interleaved in the queue
@@ -180,77 +180,6 @@ __device__ __forceinline__ int num_kv_blocks(const Params& p, int qb, int t, boo
     if (!causal) return p.num_kblocks;
     const int last = qb * (kUnitRows / kBlockN) + t;  // the diagonal block
     return min(p.num_kblocks, last + 1);
-}
-
-// One block of the online softmax for this thread's row: x_c = s_c * slv - m
-// (log2 units), p_c = 2^x_c packed to bf16 pairs, and two row sums -- in fp32
-// (for lse) and of the bf16-rounded p that enters P V (for normalising O, so
-// that O = sum(p v) / sum(p) with the same p on both sides).
-template <bool kPoly>
-__device__ __forceinline__ void exp_block(const float (&s)[kBlockN], float slv, float m_use,
-                                          uint32_t (&pk)[kBlockN / 2], float& sum, float& sum_bf16) {
-    float a[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-    float b[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-    const float neg_m = -m_use;
-#pragma unroll
-    for (int pi = 0; pi < kBlockN / 2; ++pi) {
-        float x0, x1, p0, p1;
-        if (kPackedF32x2) {
-            ptx::fma2(x0, x1, s[2 * pi], s[2 * pi + 1], slv, slv, neg_m, neg_m);
-        } else {
-            x0 = fmaf(s[2 * pi], slv, neg_m);
-            x1 = fmaf(s[2 * pi + 1], slv, neg_m);
-        }
-        if (kPoly && (pi & 7) < kPolyPairsPer8) {
-            ptx::exp2_poly2(p0, p1, x0, x1);
-        } else {
-            p0 = ptx::ex2(x0);
-            p1 = ptx::ex2(x1);
-        }
-        pk[pi] = ptx::pack_bf16x2(p0, p1);
-        if (kPackedF32x2) {
-            ptx::add2(a[pi & 3][0], a[pi & 3][1], a[pi & 3][0], a[pi & 3][1], p0, p1);
-        } else {
-            a[pi & 3][0] += p0;
-            a[pi & 3][1] += p1;
-        }
-        if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[pi & 1][0], b[pi & 1][1], pk[pi]);
-    }
-    sum = ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
-    sum_bf16 = kRowsumBf16 ? (b[0][0] + b[0][1]) + (b[1][0] + b[1][1]) : sum;
-}
-
-#ifndef FA_MAX_CHAINS
-#define FA_MAX_CHAINS 16
-#endif
-// Row max (or min) of 128 values: independent chains of three-input ops over
-// interleaved columns, then a three-way tree.
-template <bool kMax>
-__device__ __forceinline__ float reduce_row(const float (&s)[kBlockN]) {
-    constexpr int kChains = FA_MAX_CHAINS;             // 8 or 16
-    constexpr int kPer = kBlockN / kChains;             // elements per chain (16 or 8)
-    auto op3 = [](float a, float b, float c) { return kMax ? ptx::max3(a, b, c) : ptx::min3(a, b, c); };
-    auto op2 = [](float a, float b) { return kMax ? fmaxf(a, b) : fminf(a, b); };
-    float r[kChains];
-#pragma unroll
-    for (int i = 0; i < kChains; ++i) {
-        float acc = op3(s[i], s[i + kChains], s[i + 2 * kChains]);
-#pragma unroll
-        for (int e = 3; e + 1 < kPer; e += 2) acc = op3(acc, s[i + e * kChains], s[i + (e + 1) * kChains]);
-        if (kPer % 2 == 0) acc = op2(acc, s[i + (kPer - 1) * kChains]);
-        r[i] = acc;
-    }
-    // tree over the chains
-#pragma unroll
-    for (int w = kChains; w > 1;) {
-        const int n3 = w / 3, rem = w % 3;
-#pragma unroll
-        for (int i = 0; i < n3; ++i) r[i] = op3(r[3 * i], r[3 * i + 1], r[3 * i + 2]);
-        if (rem == 1) r[n3] = r[3 * n3];
-        if (rem == 2) r[n3] = op2(r[3 * n3], r[3 * n3 + 1]);
-        w = n3 + (rem ? 1 : 0);
-    }
-    return r[0];
 }
 
 // Max (or min) of each of this thread's two rows (64 values in the .16x256b
@@ -597,78 +526,102 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_phase ^= 1;
                 ptx::tc_fence_after_sync();
 
-                uint32_t sr[64];
-                ptx::tmem_ld16x256b_x16_wait(tmem_s, sr);
-                float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
-
                 const int key0 = j * kBlockN;
                 const bool need_mask = (key0 + kBlockN > p.n) || (kCausal && key0 + kBlockN - 1 > tile_row0);
-                float slv = sl;
-                if (need_mask) {
-                    // Masked block (diagonal or ragged tail): scores to log2 units
-                    // and masked keys to -inf, whatever the sign of the scale.
-                    const int lim0 = kCausal ? min(p.n - 1, row0) : (p.n - 1);
-                    const int lim1 = kCausal ? min(p.n - 1, row1) : (p.n - 1);
+                const float slv = need_mask ? 1.f : sl;  // masked blocks are pre-scaled
+                // Scores of this block into registers (masked keys to -inf,
+                // scaled to log2 units, whatever the sign of the scale).
+                uint32_t sr[64];
+                float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
+                auto load_scores = [&]() {
+                    ptx::tmem_ld16x256b_x16_wait(tmem_s, sr);
+                    if (need_mask) {
+                        const int lim0 = kCausal ? min(p.n - 1, row0) : (p.n - 1);
+                        const int lim1 = kCausal ? min(p.n - 1, row1) : (p.n - 1);
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
+                        for (int k = 0; k < 16; ++k)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int key = key0 + 8 * k + 2 * qc + (i & 1);
-                            const int lim = (i < 2) ? lim0 : lim1;
-                            s[4 * k + i] = (key <= lim) ? s[4 * k + i] * sl : -INFINITY;
-                        }
-                    slv = 1.f;
-                }
-                // row max (or min for a negative scale) over this thread's 32
-                // values per row, then across the quad
-                float mx[2];
-                if (slv >= 0.f)
-                    quad_row_extreme<true>(s, mx);
-                else
-                    quad_row_extreme<false>(s, mx);
-                mx[0] *= slv;
-                mx[1] *= slv;
-
-                // Online softmax update per row: raise the running max only
-                // when it grows by more than the threshold (the result is exact
-                // either way: O and l always share the same m).
-                float alpha[2] = {1.f, 1.f}, neg_m[2];
-                bool rescale_o = false;
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    if (j == 0) {
-                        m_run[r] = mx[r];
-                    } else if (mx[r] > m_run[r] + kRescaleThreshold) {
-                        alpha[r] = ptx::ex2(m_run[r] - mx[r]);
-                        m_run[r] = mx[r];
-                        rescale_o = true;
+                            for (int i = 0; i < 4; ++i) {
+                                const int key = key0 + 8 * k + 2 * qc + (i & 1);
+                                const int lim = (i < 2) ? lim0 : lim1;
+                                s[4 * k + i] = (key <= lim) ? s[4 * k + i] * sl : -INFINITY;
+                            }
                     }
-                    neg_m[r] = (m_run[r] == -INFINITY) ? 0.f : -m_run[r];
-                }
-
+                };
+                // Exact row max (in log2 units), completed across the quad.
+                auto block_max = [&](float (&mx)[2]) {
+                    if (slv >= 0.f)
+                        quad_row_extreme<true>(s, mx);
+                    else
+                        quad_row_extreme<false>(s, mx);
+                    mx[0] *= slv;
+                    mx[1] *= slv;
+                };
                 // p = 2^(s * slv - m): packed bf16 pairs, pk[2k] for r0 and
                 // pk[2k + 1] for r1 in chunk k (the .16x128b store order), and
-                // both row sums.  Unmasked blocks send part of the pairs through
-                // the polynomial on the FMA pipe.
+                // this thread's share of both row sums.
                 uint32_t pk[32];
-                float a[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-                float b[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                float a[2][2], b[2][2];
+                auto exponentiate = [&](const float (&neg_m)[2]) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
+                    for (int r = 0; r < 2; ++r) a[r][0] = a[r][1] = b[r][0] = b[r][1] = 0.f;
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        float x0, x1, p0, p1;
-                        ptx::fma2(x0, x1, s[4 * k + 2 * r], s[4 * k + 2 * r + 1], slv, slv, neg_m[r], neg_m[r]);
-                        if (!need_mask && ((2 * k + r) & 7) < kPolyPairsPer8) {
-                            ptx::exp2_poly2(p0, p1, x0, x1);
-                        } else {
-                            p0 = ptx::ex2(x0);
-                            p1 = ptx::ex2(x1);
+                    for (int k = 0; k < 16; ++k) {
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            float x0, x1, p0, p1;
+                            ptx::fma2(x0, x1, s[4 * k + 2 * r], s[4 * k + 2 * r + 1], slv, slv, neg_m[r], neg_m[r]);
+                            if (!need_mask && ((2 * k + r) & 7) < kPolyPairsPer8) {
+                                ptx::exp2_poly2(p0, p1, x0, x1);
+                            } else {
+                                p0 = ptx::ex2(x0);
+                                p1 = ptx::ex2(x1);
+                            }
+                            const uint32_t v = ptx::pack_bf16x2(p0, p1);
+                            pk[2 * k + r] = v;
+                            ptx::add2(a[r][0], a[r][1], a[r][0], a[r][1], p0, p1);
+                            if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[r][0], b[r][1], v);
                         }
-                        const uint32_t v = ptx::pack_bf16x2(p0, p1);
-                        pk[2 * k + r] = v;
-                        ptx::add2(a[r][0], a[r][1], a[r][0], a[r][1], p0, p1);
-                        if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[r][0], b[r][1], v);
+                    }
+                };
+                auto neg_of = [](float m) { return (m == -INFINITY) ? 0.f : -m; };
+
+                // Online softmax.  The first block of a unit sets the running
+                // max exactly.  Later blocks exponentiate against the running
+                // max as it stands and only check that no value exceeds
+                // kStaleMaxBound (a value above it makes this thread's share of
+                // a row sum exceed it); when one does -- the scores grew far past
+                // everything seen so far -- the block is redone against its
+                // exact max and O and l are rescaled.  O and l always share the
+                // same m, so the result does not depend on how stale m is.
+                load_scores();
+                float alpha[2] = {1.f, 1.f};
+                bool rescale_o = false;
+                if (j == 0) {
+                    float mx[2];
+                    block_max(mx);
+                    m_run[0] = mx[0];
+                    m_run[1] = mx[1];
+                    const float nm[2] = {neg_of(m_run[0]), neg_of(m_run[1])};
+                    exponentiate(nm);
+                } else {
+                    const float nm[2] = {neg_of(m_run[0]), neg_of(m_run[1])};
+                    exponentiate(nm);
+                    const bool big = (a[0][0] + a[0][1] > kStaleMaxBound) || (a[1][0] + a[1][1] > kStaleMaxBound);
+                    if (__any_sync(0xffffffffu, big)) {
+                        load_scores();  // P has not been stored: S is still in TMEM
+                        float mx[2];
+                        block_max(mx);
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            if (mx[r] > m_run[r]) {
+                                alpha[r] = ptx::ex2(m_run[r] - mx[r]);
+                                m_run[r] = mx[r];
+                                rescale_o = true;
+                            }
+                        }
+                        const float nm2[2] = {neg_of(m_run[0]), neg_of(m_run[1])};
+                        exponentiate(nm2);
                     }
                 }
 #pragma unroll
