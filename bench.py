@@ -67,7 +67,7 @@ def measured_peaks():
 
 def kernel_digest() -> str:
     from tiled_exact_attention_fa_b200 import build as fb
-    return fb._inputs_digest()
+    return fb.code_digest()
 
 
 def traffic_from_profile(w: W.Workload):

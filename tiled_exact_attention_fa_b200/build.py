@@ -11,6 +11,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -41,6 +42,23 @@ def _inputs_digest() -> str:
             if name.endswith((".cu", ".cuh", ".h")):
                 with open(os.path.join(d, name), "rb") as f:
                     h.update(name.encode() + f.read())
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()
+
+
+_TOKENS = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'', re.S)
+
+
+def code_digest() -> str:
+    """Digest of the library's code with comments and layout removed: it
+    changes when the compiled code can change, not when a comment does."""
+    h = hashlib.sha1()
+    for d in (CSRC, INCLUDE):
+        for name in sorted(os.listdir(d)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                with open(os.path.join(d, name)) as f:
+                    text = _TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), f.read())
+                h.update(name.encode() + " ".join(text.split()).encode())
     h.update(" ".join(ARCH + FLAGS).encode())
     return h.hexdigest()
 

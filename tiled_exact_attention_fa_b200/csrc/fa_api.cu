@@ -56,6 +56,8 @@ struct DeviceState {
 };
 
 constexpr int kMaxDevices = 64;
+// set by fa_test_skip_one_arrival; consumed by the next bf16 launch of fa_fwd
+std::atomic<int> g_skip_one_arrival{0};
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -138,6 +140,7 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
     p.num_units = p.bh * p.num_qblocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
     kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
     cudaError_t e = cudaGetLastError();
@@ -176,6 +179,11 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
 }  // namespace
 
 extern "C" {
+
+int fa_test_skip_one_arrival(void) {
+    g_skip_one_arrival.store(1);
+    return FA_OK;
+}
 
 int fa_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
     g_last_error.clear();
@@ -367,6 +375,7 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
     p.num_units = p.bh * p.num_qblocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.skip_one_arrival = 0;
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
     kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();

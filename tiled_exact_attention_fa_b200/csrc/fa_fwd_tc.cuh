@@ -17,20 +17,20 @@
 //     heads together (their K/V stay in L2) and, under the causal mask, runs
 //     each group's heaviest query blocks first (Chapter 15, "FlashAttention
 //     Evolution": work partitioning, persistent kernels);
-//   * warp 9 is the TMA producer: it takes the next unit from the queue,
+//   * warp 17 is the TMA producer: it takes the next unit from the queue,
 //     publishes it to the CTA through a shared-memory ring, loads the unit's
 //     two Q tiles once and streams K_j, V_j through a ring of 128-row
 //     shared-memory slots, all 128-byte swizzled;
-//   * warp 8 issues tcgen05.mma from one thread: S_t = Q_t K_j^T into tensor
-//     memory (TMEM), then O_t += P_t V_j with P_t read from TMEM;
-//   * warps 0-3 and 4-7 are the softmax warpgroups for the unit's two query
-//     tiles (t = 0, 1), one query row per thread: they read S_t from TMEM,
-//     update m and l, write P_t (bf16) back over S_t, rescale O_t in TMEM when
-//     the max grows past a threshold, and at the end normalise O_t and store
-//     O and lse.  While one warpgroup exponentiates, the tensor core works on
-//     the other tile.  Part of the exponentials run as a cubic polynomial on
-//     the FMA pipe, because at d = 128 the special-function unit alone would
-//     take as long as the tensor core.
+//   * warp 16 issues tcgen05.mma from one elected lane: S_t = Q_t K_j^T into
+//     tensor memory (TMEM), then O_t += P_t V_j with P_t read from TMEM;
+//   * warps 0-7 and 8-15 are the softmax warps of the unit's two query tiles
+//     (t = 0, 1), two warps per TMEM lane quarter, so a quad of threads owns
+//     two rows: they read S_t from TMEM, update m and l, write P_t (bf16)
+//     back over S_t, rescale O_t in TMEM when a block outgrows the running
+//     max, and at the end normalise O_t and store O and lse.  While one
+//     tile's warps exponentiate, the tensor core works on the other tile.
+//     At d = 128 the exponentials on the special-function unit take about as
+//     long as the tile's MMAs, so they are the co-limit of the kernel.
 //   * Causal: KV blocks entirely above the diagonal are never loaded or
 //     multiplied; only the diagonal block is masked.
 //
@@ -81,6 +81,10 @@ constexpr int kHeadGroup = 8;               // heads whose units are interleaved
 #ifndef FA_PACKED_F32X2
 #define FA_PACKED_F32X2 1
 #endif
+#ifndef FA_EARLY_K
+#define FA_EARLY_K 1
+#endif
+constexpr bool kEarlyK = FA_EARLY_K != 0;             // acquire K_{j+1} before waiting for P_0(j)
 constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;  // of every 8 column pairs, this many use exp2_poly2
 constexpr bool kRowsumBf16 = FA_ROWSUM_BF16 != 0;   // normalise O by the sum of the bf16-rounded P
 constexpr bool kPackedF32x2 = FA_PACKED_F32X2 != 0; // packed two-lane fp32 FMA/ADD
@@ -117,6 +121,7 @@ struct Params {
     int num_kblocks;     // ceil(N / 128)
     int num_units;       // bh * num_qblocks
     float scale_log2;    // scale * log2(e)
+    int skip_one_arrival;  // test hook: CTA 0 never loads its first Q tile (one wait runs out)
 };
 
 struct Sync {
@@ -310,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, wait_bar(sync, q_empty(t), (it & 1) ^ 1));
                 if (!ok) break;
                 const uint32_t dst = base + L::kQOff + t * L::kTileBytes;
+                if (p.skip_one_arrival && blockIdx.x == 0 && it == 0 && t == 0) continue;
                 q_issued[t] = (it & 1) + 1;
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
@@ -436,9 +442,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             commit(kv_empty(sk));
 
             for (int j = 0; j < n1 && ok; ++j) {
+                // V_j and K_{j+1} are waited for before P_0(j), so that PV_0(j)
+                // and S_0(j+1) go to the tensor core back to back.
                 next_slot(sv, pv);
                 ok = wait_all(kv_full(sv), pv);
                 if (!ok) break;
+                const bool more = j + 1 < n1;
+                if (more && kEarlyK) {
+                    next_slot(sk, pk);
+                    ok = wait_all(kv_full(sk), pk);
+                    if (!ok) break;
+                }
                 if (j < n0) {
                     ok = wait_all(p_full(0), p_phase[0]);
                     if (!ok) break;
@@ -447,8 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issue_pv(0, sv, j > 0);
                     if (j == n0 - 1) commit(o_full(0));
                 }
-                const bool more = j + 1 < n1;
-                if (more) {
+                if (more && !kEarlyK) {
                     next_slot(sk, pk);
                     ok = wait_all(kv_full(sk), pk);
                     if (!ok) break;
