@@ -34,7 +34,7 @@ def emulate(x):
     """exp2_poly2's steps in numpy float32, in the kernel's order."""
     c0, c1, c2, c3 = (np.float32(c) for c in header_constants())
     magic = np.float32(12582912.0)
-    x = np.maximum(np.asarray(x, np.float32), np.float32(-125.0))
+    x = np.minimum(np.maximum(np.asarray(x, np.float32), np.float32(-125.0)), np.float32(127.0))
     t = (x + magic).astype(np.float32)
     r = (t - magic).astype(np.float32)
     f = (x - r).astype(np.float32)  # exact (Sterbenz), as the fused form is
@@ -73,20 +73,31 @@ def test_clamp_below_range():
     assert np.all(y > 0) and np.all(y < 2.0 ** -124)
 
 
+def test_clamp_above_range():
+    # values the softmax must see as "far too large" (so that the block is
+    # redone against its exact max): finite, at least 2^126, never wrapped
+    with np.errstate(over="ignore"):
+        y = emulate(np.array([126.6, 127.0, 127.6, 128.0, 200.0, 1e30, np.inf], np.float32))
+    assert np.all(np.isfinite(y)) and np.all(y >= 2.0 ** 126), y
+
+
 @pytest.mark.gpu
 def test_device_routine_against_cuda_exp2():
     import tiled_exact_attention_fa_b200 as fa
     from tiled_exact_attention_fa_b200 import build as fb
     fb.build()
     x = torch.linspace(-120.0, 8.0, 1_000_001, device="cuda", dtype=torch.float32)
+    x = torch.cat([x, torch.tensor([127.0, 128.0, 200.0, float("inf"), -1000.0, float("-inf")], device="cuda")])
     y = torch.empty_like(x)
     rc = fa.library().fa_test_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(),
                                           torch.cuda.current_stream().cuda_stream)
     assert rc == 0
     torch.cuda.synchronize()
-    ref = torch.exp2(x)  # CUDA's exp2f
-    rel = (y.double() / ref.double() - 1).abs().max().item()
+    ref = torch.exp2(x[:-6])  # CUDA's exp2f
+    rel = (y[:-6].double() / ref.double() - 1).abs().max().item()
     assert rel < BOUND, rel
+    tail = y[-6:].cpu()
+    assert torch.isfinite(tail).all() and (tail[:4] >= 2.0 ** 126).all() and (tail[4:] > 0).all()
     # and the device result matches the float32 emulation of the same steps
     # (fp64-then-fp32 rounding of the fused steps can differ by one ulp on ties)
     got = y.cpu().numpy().view(np.int32).astype(np.int64)

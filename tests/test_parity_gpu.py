@@ -212,3 +212,21 @@ def test_growing_scores_take_the_slow_path(d, causal):
     v = torch.randn(1, 2, N, d, generator=g)
     q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
     check_against_oracle(q, k, v, 1.0 / 8.0, causal, strict_raw=False)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("jump_at", [64, 128, 192, 320])
+def test_score_jump_inside_a_block(d, jump_at):
+    # Every query scores keys >= jump_at about 30 log2-units above the keys
+    # before them.  A jump inside the first KV block is absorbed by the exact
+    # first-block max; a jump at the start (second) half of a later block makes
+    # the kernel redo that half and rescale O and l -- for the second half,
+    # after the first half's P V has already been issued.
+    N = 512
+    g = torch.Generator().manual_seed(67)
+    q = torch.ones(1, 2, N, d)
+    level = torch.where(torch.arange(N) >= jump_at, 30.0 * math.log(2) * 8 / d, 0.0).view(1, 1, N, 1)
+    k = level + 0.02 * torch.randn(1, 2, N, d, generator=g)
+    v = torch.randn(1, 2, N, d, generator=g)
+    q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
+    check_against_oracle(q, k, v, 1.0 / 8.0, False, strict_raw=False)

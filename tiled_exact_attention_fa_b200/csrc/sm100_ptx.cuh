@@ -345,8 +345,11 @@ constexpr float kExp2C3 = 0x1.c3f76p-5f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
 
 __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
+    // x is clamped to [-125, 127], where round(x) + the exponent of the
+    // polynomial's value stays a normal fp32 exponent: a tiny positive value
+    // below, a huge finite one (>= 2^126) above.
+    x0 = fminf(fmaxf(x0, -125.f), 127.f);
+    x1 = fminf(fmaxf(x1, -125.f), 127.f);
     float t0, t1, r0, r1, f0, f1, p0, p1;
     add2(t0, t1, x0, x1, kRoundMagic, kRoundMagic);      // low mantissa bits hold round(x)
     add2(r0, r1, t0, t1, -kRoundMagic, -kRoundMagic);    // round(x), exact
