@@ -303,7 +303,7 @@ def run_ours(a, w: W.Workload):
         line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                        "h2d_bytes_per_step": in_bytes,
                        "d2h_bytes_per_step": o.numel() * o.element_size() + lse.numel() * 4,
-                       "api": "tiled_exact_attention_fa_b200.forward(host pinned tensors, out=host pinned)"}
+                       "api": "tiled_exact_attention_fa_b200.forward(host pinned tensors, out=host pinned) -> fa_fwd_host (C ABI; chunked, pipelined copies)"}
         if "value" not in line:
             line["value"] = line["e2e"]["value"]
 

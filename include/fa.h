@@ -114,6 +114,31 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
                    float scale, int causal, int dtype, void* stream);
 
 /*
+ * fa_fwd_host -- fa_fwd on buffers in host memory: the same operation,
+ * arguments, layouts, results and errors, but q, k, v, o and lse may be host
+ * pointers (page-locked memory, e.g. from cudaHostAlloc, for the copies to
+ * run asynchronously; pageable memory works but its copies are synchronous).
+ * Device pointers are accepted too (copies are direction-inferred).  No
+ * alignment is required.  The pages have no counterpart: this is the path a
+ * caller with host-resident data uses, and the one end-to-end timings go
+ * through.
+ *
+ * The heads are processed in chunks (about eight per call) that flow through
+ * three device staging buffers and three internal streams: while one chunk
+ * is copied in, the kernel runs on the previous one and the one before is
+ * copied out.  The staging buffers are allocated on first use on each device
+ * and grown when a call needs more; they are kept until process exit.  Work
+ * starts after everything already enqueued on `stream` and `stream` waits for
+ * the last copy-out, so synchronising `stream` (or fa_check_device_status)
+ * makes o and lse valid on the host; the host buffers must stay valid until
+ * then.  Concurrent calls on one device are serialised while they enqueue and
+ * then run in order on the device.
+ */
+int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                int64_t B, int64_t H, int64_t N, int64_t d,
+                float scale, int causal, int dtype, void* stream);
+
+/*
  * fa_check_device_status -- synchronise `stream`, then read and clear the
  * library's device status word for the current device.  Returns FA_OK,
  * FA_ERR_DEVICE_TIMEOUT when a kernel launched by this library gave up on a

@@ -106,3 +106,30 @@ def test_no_gpu_is_an_error_not_a_fallback(lib):
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises((RuntimeError, AssertionError)):
         fa.forward(q, q, q)
+
+
+def call_host(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,
+              scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16):
+    return lib.fa_fwd_host(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, None)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(lse=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(N=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(dtype=7), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(o=A + 16), fa.FA_ERR_INVALID_ARGUMENT),          # o overlaps q
+    (dict(lse=A + 3 * NB + 64), fa.FA_ERR_INVALID_ARGUMENT),  # lse inside o
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+])
+def test_host_entry_rejected_before_cuda(lib, kwargs, code):
+    assert call_host(lib, **kwargs) == code
+    assert lib.fa_last_error().decode() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_host_entry_needs_no_alignment_but_a_gpu(lib):
+    # host buffers need no alignment: a misaligned q passes the checks and the
+    # call then fails on the missing GPU
+    assert call_host(lib, q=A + 2) == fa.FA_ERR_CUDA

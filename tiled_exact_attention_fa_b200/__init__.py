@@ -34,6 +34,8 @@ _SIGNATURES = {
                [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "fa_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
+                    [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
@@ -90,19 +92,10 @@ def forward_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                  lse: torch.Tensor, *, scale: float | None = None, causal: bool = False,
                  stream: torch.cuda.Stream | None = None) -> None:
     """Run the forward into caller-provided CUDA tensors o [B,H,N,d] and lse [B,H,N] fp32."""
-    if q.dtype not in _DTYPES or not (q.dtype == k.dtype == v.dtype == o.dtype):
-        raise TypeError("q, k, v, o must all be bf16 or all fp32")
-    if lse.dtype != torch.float32:
-        raise TypeError("lse must be fp32")
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
-        raise ValueError("q, k, v, o must share one [B, H, N, d] shape")
-    if lse.shape != q.shape[:3]:
-        raise ValueError("lse must be [B, H, N]")
+    _check_qkv(q, k, v, o, lse)
     for t in (q, k, v, o, lse):
         if not t.is_cuda:
             raise ValueError("forward_into needs CUDA tensors")
-        if not t.is_contiguous():
-            raise ValueError("tensors must be contiguous")
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -112,33 +105,59 @@ def forward_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                       B, H, N, d, float(scale), causal, _DTYPES[q.dtype], s))
 
 
+def _check_qkv(q, k, v, o, lse):
+    if q.dtype not in _DTYPES or not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise TypeError("q, k, v, o must all be bf16 or all fp32")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be fp32")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
+        raise ValueError("q, k, v, o must share one [B, H, N, d] shape")
+    if lse.shape != q.shape[:3]:
+        raise ValueError("lse must be [B, H, N]")
+    for t in (q, k, v, o, lse):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def forward_host_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                      lse: torch.Tensor, *, scale: float | None = None, causal: bool = False,
+                      stream: torch.cuda.Stream | None = None) -> None:
+    """fa_fwd_host on host tensors (pinned for asynchronous copies) on the
+    current CUDA device; o and lse are valid once `stream` (default: the
+    current stream) has been synchronised."""
+    _check_qkv(q, k, v, o, lse)
+    if any(t.is_cuda for t in (q, k, v, o, lse)):
+        raise ValueError("forward_host_into takes host tensors")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(int(library().fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                     B, H, N, d, float(scale), int(causal), _DTYPES[q.dtype], s)))
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
             causal: bool = False, out: tuple[torch.Tensor, torch.Tensor] | None = None):
     """Exact attention forward.  Returns (o, lse).
 
     q, k, v: [B, H, N, d] bf16 or fp32, d in {64, 128}.  CUDA tensors give CUDA
-    outputs.  Host tensors are copied to the current CUDA device (pinned memory
-    makes the copies asynchronous), computed there, and the outputs are copied
-    back into host tensors -- `out=(o, lse)` if given (pinned, preallocated),
-    else new pinned tensors -- before the call returns.
+    outputs.  Host tensors go through fa_fwd_host (chunks of heads copied in,
+    computed and copied out in a pipeline on the current CUDA device) into
+    host tensors -- `out=(o, lse)` if given, else new pinned tensors -- that
+    are complete when the call returns.
     """
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        q, k, v = (x.to(dev, non_blocking=True) for x in (q, k, v))
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if not q.is_cuda:
+        if out is None:
+            out = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True),
+                   torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True))
+        stream = torch.cuda.current_stream()
+        forward_host_into(q, k, v, out[0], out[1], scale=scale, causal=causal, stream=stream)
+        stream.synchronize()
+        return out
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     forward_into(q, k, v, o, lse, scale=scale, causal=causal)
-    if host:
-        if out is None:
-            out = (torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
-                   torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True))
-        o_h, lse_h = out
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        return o_h, lse_h
     if out is not None:
         out[0].copy_(o)
         out[1].copy_(lse)

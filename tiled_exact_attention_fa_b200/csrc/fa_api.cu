@@ -166,6 +166,66 @@ int launch_f32(const void* q, const void* k, const void* v, void* o, float* lse,
     return FA_OK;
 }
 
+// Argument checks shared by the entry points; all run before any CUDA call.
+struct Sizes {
+    int64_t bh = 0;
+    int64_t elem = 0;
+    size_t tensor_bytes = 0;
+    size_t lse_bytes = 0;
+};
+
+int check_args(const void* q, const void* k, const void* v, const void* o, const float* lse, int64_t B,
+               int64_t H, int64_t N, int64_t d, float scale, int dtype, bool device_pointers, Sizes* z) {
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    const int64_t bh = B * H;
+    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
+    const int64_t units = bh * ((N + 255) / 256);
+    if (units > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
+    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
+    if (bh > (int64_t{1} << 62) / (N * d * elem)) return fail(FA_ERR_INVALID_ARGUMENT, "tensor size overflows");
+    const size_t tensor_bytes = static_cast<size_t>(bh * N * d * elem);
+    const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
+    auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (device_pointers) {
+        if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16))
+            return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+        if (misaligned(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    }
+    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
+        overlaps(o, tensor_bytes, v, tensor_bytes) || overlaps(o, tensor_bytes, lse, lse_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
+    if (overlaps(lse, lse_bytes, q, tensor_bytes) || overlaps(lse, lse_bytes, k, tensor_bytes) ||
+        overlaps(lse, lse_bytes, v, tensor_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
+    z->bh = bh;
+    z->elem = elem;
+    z->tensor_bytes = tensor_bytes;
+    z->lse_bytes = lse_bytes;
+    return FA_OK;
+}
+
+// Kernel choice and launch on `s` for bh heads of N rows (device pointers).
+int dispatch(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh,
+             int64_t N, int64_t d, float scale, bool c, int dtype, cudaStream_t s) {
+    if (dtype == FA_DTYPE_BF16) {
+        if (st->cc_major != 10)
+            return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
+        if (d == 128) return c ? launch_bf16<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
+                               : launch_bf16<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
+        return c ? launch_bf16<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
+                 : launch_bf16<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
+    }
+    if (d == 128) return c ? launch_f32<128, true>(q, k, v, o, lse, bh, N, scale, s)
+                           : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
+    return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
+             : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+}
+
 __global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
     const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
     if (i >= n) return;
@@ -215,50 +275,12 @@ const char* fa_last_error(void) { return g_last_error.c_str(); }
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t N,
            int64_t d, float scale, int causal, int dtype, void* stream) {
     g_last_error.clear();
-    // ---- argument checks: all before any CUDA call
-    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
-    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
-    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
-    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
-    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
-    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
-    const int64_t bh = B * H;
-    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
-    const int64_t units = bh * ((N + 255) / 256);
-    if (units > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
-    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
-    if (bh > (int64_t{1} << 62) / (N * d * elem)) return fail(FA_ERR_INVALID_ARGUMENT, "tensor size overflows");
-    const size_t tensor_bytes = static_cast<size_t>(bh * N * d * elem);
-    const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
-    auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
-    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16))
-        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
-    if (misaligned(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
-    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
-        overlaps(o, tensor_bytes, v, tensor_bytes) || overlaps(o, tensor_bytes, lse, lse_bytes))
-        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
-    if (overlaps(lse, lse_bytes, q, tensor_bytes) || overlaps(lse, lse_bytes, k, tensor_bytes) ||
-        overlaps(lse, lse_bytes, v, tensor_bytes))
-        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
-
-    // ---- device set-up (first call per device) and dispatch
-    DeviceState* st = nullptr;
-    int rc = device_state(&st);
+    Sizes z;
+    int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, dtype, true, &z);
     if (rc != FA_OK) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool c = causal != 0;
-    if (dtype == FA_DTYPE_BF16) {
-        if (st->cc_major != 10)
-            return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
-        if (d == 128) return c ? launch_bf16<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
-                               : launch_bf16<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
-        return c ? launch_bf16<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
-                 : launch_bf16<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
-    }
-    if (d == 128) return c ? launch_f32<128, true>(q, k, v, o, lse, bh, N, scale, s)
-                           : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
-    return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
-             : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    return dispatch(st, q, k, v, o, lse, z.bh, N, d, scale, causal != 0, dtype, static_cast<cudaStream_t>(stream));
 }
 
 int fa_check_device_status(void* stream) {
@@ -437,4 +459,131 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
                            : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
     return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
              : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+}
+
+// ---------------------------------------------------------------------------
+// fa_fwd_host: the forward on host buffers.  The heads are processed in
+// chunks through three device staging buffers on three internal streams, so
+// that the copy-in of one chunk, the kernel of the previous one and the
+// copy-out of the one before run at the same time (host-to-device and
+// device-to-host copies use separate copy engines).  For pinned host memory
+// the whole call then costs about the longer of the two copy directions
+// instead of their sum plus the kernel.
+namespace {
+
+constexpr int kPipeBuffers = 3;
+constexpr int64_t kPipeChunks = 8;  // target number of chunks per call
+
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+    cudaEvent_t ev_entry = nullptr, ev_done = nullptr;
+    cudaEvent_t ev_in[kPipeBuffers] = {}, ev_comp[kPipeBuffers] = {}, ev_free[kPipeBuffers] = {};
+    char* buf[kPipeBuffers] = {};
+    size_t buf_bytes = 0;
+    std::mutex mu;  // one call at a time enqueues on this device's pipeline
+};
+HostPipe g_pipe[kMaxDevices];
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int pipe_setup(HostPipe& pp) {
+    if (pp.ready) return FA_OK;
+    cudaError_t e;
+    for (cudaStream_t* s : {&pp.s_in, &pp.s_comp, &pp.s_out})
+        if ((e = cudaStreamCreateWithFlags(s, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithFlags");
+    if ((e = cudaEventCreateWithFlags(&pp.ev_entry, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&pp.ev_done, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventCreateWithFlags");
+    for (int b = 0; b < kPipeBuffers; ++b)
+        for (cudaEvent_t* ev : {&pp.ev_in[b], &pp.ev_comp[b], &pp.ev_free[b]})
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(e, "cudaEventCreateWithFlags");
+    pp.ready = true;
+    return FA_OK;
+}
+
+// Staging buffers of at least `bytes` each; growing waits for the pipeline
+// to drain first, since queued work may still use the old buffers.
+int pipe_reserve(HostPipe& pp, size_t bytes) {
+    if (pp.buf_bytes >= bytes) return FA_OK;
+    cudaError_t e;
+    for (cudaStream_t s : {pp.s_in, pp.s_comp, pp.s_out})
+        if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    for (int b = 0; b < kPipeBuffers; ++b) {
+        if (pp.buf[b] && (e = cudaFree(pp.buf[b])) != cudaSuccess) return cuda_fail(e, "cudaFree(staging)");
+        pp.buf[b] = nullptr;
+    }
+    pp.buf_bytes = 0;
+    for (int b = 0; b < kPipeBuffers; ++b)
+        if ((e = cudaMalloc(&pp.buf[b], bytes)) != cudaSuccess) return cuda_fail(e, "cudaMalloc(staging)");
+    pp.buf_bytes = bytes;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                           int64_t N, int64_t d, float scale, int causal, int dtype, void* stream) {
+    g_last_error.clear();
+    Sizes z;
+    int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, dtype, false, &z);
+    if (rc != FA_OK) return rc;
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    HostPipe& pp = g_pipe[dev];
+    std::lock_guard<std::mutex> lock(pp.mu);
+    if ((rc = pipe_setup(pp)) != FA_OK) return rc;
+
+    const int64_t ch = (z.bh + kPipeChunks - 1) / kPipeChunks;  // heads per chunk
+    const size_t head_bytes = static_cast<size_t>(N * d * z.elem), head_lse = static_cast<size_t>(N * 4);
+    const size_t t_bytes = round_up(ch * head_bytes, 256), l_bytes = round_up(ch * head_lse, 256);
+    if ((rc = pipe_reserve(pp, 4 * t_bytes + l_bytes)) != FA_OK) return rc;
+
+    cudaStream_t caller = static_cast<cudaStream_t>(stream);
+    auto ck = [&](cudaError_t err, const char* what) { return err == cudaSuccess ? FA_OK : cuda_fail(err, what); };
+    if ((rc = ck(cudaEventRecord(pp.ev_entry, caller), "cudaEventRecord")) != FA_OK) return rc;
+    if ((rc = ck(cudaStreamWaitEvent(pp.s_in, pp.ev_entry, 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
+    const char* hq = static_cast<const char*>(q);
+    const char* hk = static_cast<const char*>(k);
+    const char* hv = static_cast<const char*>(v);
+    char* ho = static_cast<char*>(o);
+    char* hl = reinterpret_cast<char*>(lse);
+    const int64_t nchunks = (z.bh + ch - 1) / ch;
+    for (int64_t i = 0; i < nchunks; ++i) {
+        const int b = static_cast<int>(i % kPipeBuffers);
+        const int64_t h0 = i * ch, hc = (h0 + ch <= z.bh) ? ch : z.bh - h0;
+        const size_t off = static_cast<size_t>(h0) * head_bytes, nb = static_cast<size_t>(hc) * head_bytes;
+        const size_t loff = static_cast<size_t>(h0) * head_lse, lnb = static_cast<size_t>(hc) * head_lse;
+        char* dq = pp.buf[b];
+        char* dk = dq + t_bytes;
+        char* dv = dk + t_bytes;
+        char* dout = dv + t_bytes;
+        float* dl = reinterpret_cast<float*>(dout + t_bytes);
+        // copy-in once the buffer's previous chunk (of this call or an earlier
+        // one) has been copied out; an event never recorded is no wait
+        if ((rc = ck(cudaStreamWaitEvent(pp.s_in, pp.ev_free[b], 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
+        if ((rc = ck(cudaMemcpyAsync(dq, hq + off, nb, cudaMemcpyDefault, pp.s_in), "cudaMemcpyAsync(q)")) != FA_OK ||
+            (rc = ck(cudaMemcpyAsync(dk, hk + off, nb, cudaMemcpyDefault, pp.s_in), "cudaMemcpyAsync(k)")) != FA_OK ||
+            (rc = ck(cudaMemcpyAsync(dv, hv + off, nb, cudaMemcpyDefault, pp.s_in), "cudaMemcpyAsync(v)")) != FA_OK ||
+            (rc = ck(cudaEventRecord(pp.ev_in[b], pp.s_in), "cudaEventRecord")) != FA_OK)
+            return rc;
+        // the kernel on this chunk's heads
+        if ((rc = ck(cudaStreamWaitEvent(pp.s_comp, pp.ev_in[b], 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
+        if ((rc = dispatch(st, dq, dk, dv, dout, dl, hc, N, d, scale, causal != 0, dtype, pp.s_comp)) != FA_OK) return rc;
+        if ((rc = ck(cudaEventRecord(pp.ev_comp[b], pp.s_comp), "cudaEventRecord")) != FA_OK) return rc;
+        // copy-out
+        if ((rc = ck(cudaStreamWaitEvent(pp.s_out, pp.ev_comp[b], 0), "cudaStreamWaitEvent")) != FA_OK ||
+            (rc = ck(cudaMemcpyAsync(ho + off, dout, nb, cudaMemcpyDefault, pp.s_out), "cudaMemcpyAsync(o)")) != FA_OK ||
+            (rc = ck(cudaMemcpyAsync(hl + loff, dl, lnb, cudaMemcpyDefault, pp.s_out), "cudaMemcpyAsync(lse)")) != FA_OK ||
+            (rc = ck(cudaEventRecord(pp.ev_free[b], pp.s_out), "cudaEventRecord")) != FA_OK)
+            return rc;
+    }
+    // the caller's stream continues once the last copy-out is done
+    if ((rc = ck(cudaEventRecord(pp.ev_done, pp.s_out), "cudaEventRecord")) != FA_OK) return rc;
+    return ck(cudaStreamWaitEvent(caller, pp.ev_done, 0), "cudaStreamWaitEvent");
 }
