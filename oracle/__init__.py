@@ -65,6 +65,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
         ctypes.c_void_p, ctypes.c_void_p]
+    g = lib.oracle_attention_decode
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_version.restype = ctypes.c_int
     return lib
@@ -115,4 +119,28 @@ def attention_fwd(q, k, v, scale: float, causal: bool, rows=None, lib=None):
         int(bool(causal)), rows.ctypes.data, R, o.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise RuntimeError(f"oracle_attention_fwd failed with code {rc}")
+    return o, lse
+
+
+def attention_decode(q, k, v, scale: float, causal: bool, lib=None):
+    """Attention of nq new queries over nk cached keys, in fp64.
+
+    q: [B, H, nq, d]; k, v: [B, H, nk, d] (exact input values, fp32).  Query i
+    sits at position nk - nq + i; causal restricts it to keys <= that position.
+    Returns (o, lse): o is [B, H, nq, d] fp64, lse is [B, H, nq] fp64 natural log.
+    """
+    lib = lib or load()
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    if q.ndim != 4 or k.ndim != 4 or k.shape != v.shape or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be [B, H, nq, d] and k, v [B, H, nk, d]")
+    B, H, nq, d = q.shape
+    nk = k.shape[2]
+    o = np.empty((B, H, nq, d), dtype=np.float64)
+    lse = np.empty((B, H, nq), dtype=np.float64)
+    rc = lib.oracle_attention_decode(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * H, nq, nk, d,
+                                     float(scale), int(bool(causal)), o.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_decode failed with code {rc}")
     return o, lse

@@ -153,3 +153,66 @@ int oracle_attention_fwd(const float* q, const float* k, const float* v,
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * oracle_attention_decode -- the same definition for new tokens attending
+ * to a key/value cache ("FlashAttention: Tiled & Fused", card "KV Cache: Why
+ * Generation Speeds Up": past K and V are cached and each new token computes
+ * only its own).  nq new queries, nk cached keys (the new tokens' own keys
+ * are the last nq of them).  Query i sits at sequence position
+ * nk - nq + i; with causal it may use keys kj <= nk - nq + i, without it all
+ * nk keys.  Each query's full score row is materialised and softmaxed in
+ * two passes, as above.
+ *   q:    [bh][nq][d] fp32         k, v: [bh][nk][d] fp32
+ *   o:    [bh][nq][d] fp64         lse:  [bh][nq] fp64 (natural log)
+ * Returns 0 on success, -1 on bad arguments, -2 if scratch cannot be allocated.
+ */
+int oracle_attention_decode(const float* q, const float* k, const float* v,
+                            int64_t bh, int64_t nq, int64_t nk, int64_t d, double scale, int causal,
+                            double* o, double* lse) {
+    if (!q || !k || !v || !o || !lse) return -1;
+    if (bh <= 0 || nq <= 0 || nk <= 0 || d <= 0) return -1;
+    if (causal && nq > nk) return -1;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* w = (double*)malloc((size_t)nk * sizeof(double)); /* one score row */
+        if (!w) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t task = 0; task < bh * nq; ++task) {
+            if (!w) continue;
+            const int64_t h = task / nq, qi = task % nq;
+            const float* qrow = q + (h * nq + qi) * d;
+            const float* kh = k + h * nk * d;
+            const float* vh = v + h * nk * d;
+            const int64_t last = causal ? nk - nq + qi : nk - 1; /* last key this query may use */
+            /* scores of the allowed keys */
+            for (int64_t kj = 0; kj <= last; ++kj) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < d; ++t) acc += (double)qrow[t] * (double)kh[kj * d + t];
+                w[kj] = acc * scale;
+            }
+            /* softmax: the max, then the exponentials and their sum */
+            double mx = w[0];
+            for (int64_t kj = 1; kj <= last; ++kj) mx = (w[kj] > mx) ? w[kj] : mx;
+            double sum = 0.0;
+            for (int64_t kj = 0; kj <= last; ++kj) {
+                w[kj] = exp(w[kj] - mx);
+                sum += w[kj];
+            }
+            /* O = P V with P = w / sum */
+            double* orow = o + (h * nq + qi) * d;
+            for (int64_t t = 0; t < d; ++t) {
+                double acc = 0.0;
+                for (int64_t kj = 0; kj <= last; ++kj) acc += w[kj] * (double)vh[kj * d + t];
+                orow[t] = acc / sum;
+            }
+            lse[h * nq + qi] = mx + log(sum);
+        }
+        free(w);
+    }
+    return failed ? -2 : 0;
+}

@@ -266,8 +266,113 @@ def pin_torch_sdpa(lib):
         np.testing.assert_allclose(lse, lt.numpy(), rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------- decode over a key/value cache
+# New tokens attend to the cached keys ("FlashAttention: Tiled & Fused", card
+# "KV Cache: Why Generation Speeds Up"); query i of nq sits at position
+# nk - nq + i.
+
+def _dec(lib, q, k, v, scale, causal):
+    return oracle.attention_decode(q, k, v, scale, causal, lib=lib)
+
+
+def pin_decode_hand_worked(lib):
+    """One query, two cached keys, d = 1, scale = 1: q = 1, k = [0, ln 3],
+    v = [4, 8] -> weights [1/4, 3/4], o = 1 + 6 = 7, lse = ln 4 (with the fp32
+    value of ln 3 carried through)."""
+    a = float(np.float32(math.log(3.0)))
+    q = np.ones((1, 1, 1, 1), np.float32)
+    k = np.array([0.0, a], np.float32).reshape(1, 1, 2, 1)
+    v = np.array([4.0, 8.0], np.float32).reshape(1, 1, 2, 1)
+    for causal in (False, True):  # the only query is the last position: the mask changes nothing
+        o, lse = _dec(lib, q, k, v, 1.0, causal)
+        w1 = math.exp(a) / (1.0 + math.exp(a))
+        assert abs(o[0, 0, 0, 0] - (4 * (1 - w1) + 8 * w1)) < 1e-13, o
+        assert abs(o[0, 0, 0, 0] - 7.0) < 1e-6
+        assert abs(lse[0, 0, 0] - math.log(1.0 + math.exp(a))) < 1e-14
+
+
+def pin_decode_closed_forms(lib):
+    """q = 0: o_i is the mean of the keys query i may use (nk - nq + i + 1 of
+    them under the causal mask) and lse_i = ln of their count.  nk = 1: o = v_0
+    and lse = scale * q . k_0."""
+    B, H, nq, nk, d = 2, 2, 5, 23, 8
+    k = _rand((B, H, nk, d), 40)
+    v = _rand((B, H, nk, d), 41)
+    q = np.zeros((B, H, nq, d), np.float32)
+    for causal in (False, True):
+        o, lse = _dec(lib, q, k, v, 0.9, causal)
+        for i in range(nq):
+            n_allowed = nk - nq + i + 1 if causal else nk
+            np.testing.assert_allclose(o[:, :, i], v[:, :, :n_allowed].astype(np.float64).mean(axis=2),
+                                       rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lse[:, :, i], math.log(n_allowed), rtol=0, atol=1e-13)
+    q1 = _rand((B, H, 1, d), 42)
+    o, lse = _dec(lib, q1, k[:, :, :1], v[:, :, :1], 0.3, True)
+    np.testing.assert_array_equal(o[:, :, 0], v[:, :, 0].astype(np.float64))
+    want = 0.3 * np.einsum("bhd,bhd->bh", q1[:, :, 0].astype(np.float64), k[:, :, 0].astype(np.float64))
+    np.testing.assert_allclose(lse[:, :, 0], want, rtol=0, atol=1e-13)
+
+
+def pin_decode_is_the_last_rows_of_prefill(lib):
+    """The queries of a decode step are the last nq rows of the full attention
+    over the whole sequence: decoding them against the cache must give the
+    full computation's rows nk - nq .. nk - 1, causal or not."""
+    B, H, nk, d, nq = 1, 3, 70, 16, 4
+    qf = _rand((B, H, nk, d), 50)
+    k = _rand((B, H, nk, d), 51)
+    v = _rand((B, H, nk, d), 52)
+    rows = np.broadcast_to(np.arange(nk - nq, nk, dtype=np.int64), (B, H, nq))
+    for causal in (False, True):
+        o_full, lse_full = _run(lib, qf, k, v, 0.2, causal, rows=rows)
+        o, lse = _dec(lib, qf[:, :, nk - nq:], k, v, 0.2, causal)
+        np.testing.assert_allclose(o, o_full, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, lse_full, rtol=0, atol=1e-13)
+
+
+def pin_decode_future_keys_ignored(lib):
+    """Under the causal mask query i must not depend on cached keys past its
+    position nk - nq + i; without the mask it depends on all of them."""
+    B, H, nq, nk, d = 1, 2, 6, 40, 8
+    q = _rand((B, H, nq, d), 60)
+    k = _rand((B, H, nk, d), 61)
+    v = _rand((B, H, nk, d), 62)
+    o, lse = _dec(lib, q, k, v, 0.5, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, nk - nq + 1:] += 3.0  # every key after query 0's position
+    v2[:, :, nk - nq + 1:] -= 2.0
+    o2, lse2 = _dec(lib, q, k2, v2, 0.5, True)
+    np.testing.assert_array_equal(o2[:, :, 0], o[:, :, 0])
+    np.testing.assert_array_equal(lse2[:, :, 0], lse[:, :, 0])
+    assert np.abs(o2[:, :, 1:] - o[:, :, 1:]).max() > 1e-3
+    o3, _ = _dec(lib, q, k2, v2, 0.5, False)
+    o4, _ = _dec(lib, q, k, v, 0.5, False)
+    assert np.abs(o3 - o4).max() > 1e-3
+
+
+def pin_decode_torch_sdpa(lib):
+    """torch's fp64 math attention with an explicit boolean mask (query i may
+    use keys <= nk - nq + i) and the scale passed in, and torch.logsumexp."""
+    B, H, nq, nk, d = 2, 2, 7, 300, 32
+    q = _rand((B, H, nq, d), 70)
+    k = _rand((B, H, nk, d), 71)
+    v = _rand((B, H, nk, d), 72)
+    tq, tk, tv = (torch.from_numpy(x.astype(np.float64)) for x in (q, k, v))
+    pos = torch.arange(nk - nq, nk).view(nq, 1)
+    for causal in (False, True):
+        mask = (torch.arange(nk).view(1, nk) <= pos) if causal else torch.ones(nq, nk, dtype=torch.bool)
+        o_ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.17)
+        s = (tq @ tk.transpose(-1, -2)) * 0.17
+        lse_ref = torch.logsumexp(s.masked_fill(~mask, float("-inf")), dim=-1)
+        o, lse = _dec(lib, q, k, v, 0.17, causal)
+        np.testing.assert_allclose(o, o_ref.numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_ref.numpy(), rtol=0, atol=1e-12)
+
+
+DECODE_PINS = [pin_decode_hand_worked, pin_decode_closed_forms, pin_decode_is_the_last_rows_of_prefill,
+               pin_decode_future_keys_ignored, pin_decode_torch_sdpa]
+
 ALL_PINS = [
     pin_hand_worked, pin_q_zero_mean_of_v, pin_single_key, pin_causal_row0, pin_affine_v,
     pin_key_permutation, pin_future_keys_ignored, pin_softmax_shift, pin_lse_bounds,
     pin_row_subset, pin_online_ledger, pin_torch_sdpa,
-]
+] + DECODE_PINS

@@ -27,6 +27,18 @@ MUTANTS = [
      "dot += (double)q[t * n + i % n] * (double)kj[t];"),
     ("fp32_dot", "double dot = 0.0;", "float dot = 0.0f;"),
     ("max_from_first_key_only", "if (srow[j] > m) m = srow[j];", "if (j == 0) m = srow[j];"),
+    # the decode function
+    ("decode_top_left_mask", "const int64_t last = causal ? nk - nq + qi : nk - 1;",
+     "const int64_t last = causal ? qi : nk - 1;"),
+    ("decode_own_key_masked", "const int64_t last = causal ? nk - nq + qi : nk - 1;",
+     "const int64_t last = causal ? nk - nq + qi - 1 : nk - 1;"),
+    ("decode_last_key_dropped", "const int64_t last = causal ? nk - nq + qi : nk - 1;",
+     "const int64_t last = causal ? nk - nq + qi : nk - 2;"),
+    ("decode_scale_dropped", "w[kj] = acc * scale;", "w[kj] = acc;"),
+    ("decode_lse_without_max", "lse[h * nq + qi] = mx + log(sum);", "lse[h * nq + qi] = log(sum);"),
+    ("decode_not_normalised", "orow[t] = acc / sum;", "orow[t] = acc;"),
+    ("decode_v_of_key_0", "acc += w[kj] * (double)vh[kj * d + t];", "acc += w[kj] * (double)vh[t];"),
+    ("decode_query_of_head_0", "const float* qrow = q + (h * nq + qi) * d;", "const float* qrow = q + qi * d;"),
 ]
 
 
