@@ -14,6 +14,10 @@ slowest rank's.
 
 `--impl reference` times the fp64 CPU oracle (test infrastructure, the
 deliberately slow plain definition) on a bounded sample of the same workload.
+
+`--path decode` measures the generation step instead (fa_decode: new queries
+over a resident key/value cache, HBM-bound): the metric is the cache bytes
+read per second, against the measured HBM copy bandwidth.
 """
 from __future__ import annotations
 
@@ -53,6 +57,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
+    ap.add_argument("--path", default="forward", choices=["forward", "decode"])
+    ap.add_argument("--decode-workload", default=W.DECODE_HEADLINE.name, choices=sorted(W.DECODE_BY_NAME))
     return ap.parse_args()
 
 
@@ -65,12 +71,12 @@ def measured_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def kernel_digest() -> str:
+def kernel_digest(kind: str) -> str:
     from tiled_exact_attention_fa_b200 import build as fb
-    return fb.code_digest()
+    return fb.code_digest(fb.KERNEL_SOURCES[kind])
 
 
-def traffic_from_profile(w: W.Workload):
+def traffic_from_profile(w):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
     workload, or None when there is none or the kernel changed since."""
     path = os.path.join(PROFILE_DIR, f"traffic_{w.name}.json")
@@ -78,7 +84,8 @@ def traffic_from_profile(w: W.Workload):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("kernel_digest") != kernel_digest():
+    kind = "decode" if isinstance(w, W.DecodeWorkload) else "forward"
+    if d.get("kernel_digest") != kernel_digest(kind):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -318,8 +325,174 @@ def run_ours(a, w: W.Workload):
     return 0
 
 
+DECODE_METRIC = "attention decode: K/V cache bytes read per second (bf16, d=128) vs measured HBM bandwidth"
+DECODE_UNIT = "GB/s"
+
+
+def decode_config(w: W.DecodeWorkload) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "nq": w.nq, "nk": w.nk, "d": w.d, "causal": w.causal,
+            "seed": w.seed}
+
+
+def decode_cpu_sample(w: W.DecodeWorkload, seconds: float, seed: int):
+    """Time the fp64 oracle on as many heads of the workload as fit in about
+    `seconds`; returns (GB/s of cache processed, heads, elapsed s)."""
+    import oracle
+    g = torch.Generator().manual_seed(seed)
+
+    def draw(n, heads):
+        return torch.randn((1, heads, n, w.d), generator=g).to(w.dtype).float().numpy()
+
+    def run(heads):
+        q, k, v = draw(w.nq, heads), draw(w.nk, heads), draw(w.nk, heads)
+        t0 = time.perf_counter()
+        oracle.attention_decode(q, k, v, w.scale, w.causal)
+        return time.perf_counter() - t0
+
+    per_head_bytes = w.cache_bytes() / (w.B * w.H)
+    dt = run(1)
+    heads = int(max(1, min(w.B * w.H, seconds / max(dt, 1e-6))))
+    dt = run(heads)
+    return heads * per_head_bytes / dt / 1e9, heads, dt
+
+
+def run_decode_reference(a, w: W.DecodeWorkload):
+    rank, _, world = fdist.env_world()
+    if rank != 0:
+        return 0
+    import oracle
+    per_step_s = max(0.05, min(5.0, 150.0 / max(1, a.steps + a.warmup)))
+    for _ in range(a.warmup):
+        decode_cpu_sample(w, per_step_s, w.seed + 11)
+    vals, times, heads = [], [], 0
+    for i in range(a.steps):
+        gbs, heads, dt = decode_cpu_sample(w, per_step_s, w.seed + 12 + i)
+        vals.append(gbs * dt)
+        times.append(dt)
+    value = sum(vals) / sum(times)
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": decode_config(w),
+            "cpu_baseline": {"value": value, "unit": DECODE_UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"each step: {heads} heads of {w.name}"},
+            "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(a, w: W.DecodeWorkload):
+    import tiled_exact_attention_fa_b200 as fa
+
+    rank, local_rank, world = fdist.env_world()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        fdist.init("nccl", timeout_s=300)
+    legs = set(a.legs.split(","))
+    wr = W.DecodeWorkload(w.name, w.dtype, w.B, w.H, w.nq, w.nk, w.d, w.causal, w.seed + 1000 * rank)
+    q, k, v = W.make_decode_inputs(wr, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    ws = fa.decode_workspace(w.B, w.H, w.nq, w.nk, w.d, dev)
+    stream = torch.cuda.current_stream(dev)
+    esz = q.element_size()
+    alg_bytes = w.cache_bytes() + 2 * q.numel() * esz + lse.numel() * 4  # K, V, Q read; O, lse written
+
+    def step():
+        fa.decode_into(q, k, v, o, lse, scale=w.scale, causal=w.causal, workspace=ws)
+
+    for _ in range(a.warmup):
+        step()
+    fa.check_device_status()
+    line = {"metric": DECODE_METRIC, "unit": DECODE_UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic"}
+    line["config"] = dict(decode_config(w), per_rank="own seeded batch (seed + 1000*rank), no collective",
+                          l2=f"K/V cache {w.cache_bytes() / 2**30:.1f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB, no flush",
+                          bytes_per_step=alg_bytes)
+    if "kernel" in legs:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
+            fdist.barrier(dev)
+            torch.cuda.synchronize(dev)
+            start.record(stream)
+            for _ in range(a.steps):
+                step()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+            fdist.barrier(dev)
+        fa.check_device_status()
+        ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.steps
+        gbs = alg_bytes / (ms * 1e-3) / 1e9
+        _, _, hbm, peak_kind = measured_peaks()
+        line["value"] = world * gbs
+        line["ms_per_step"] = ms
+        line["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                            "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                            "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
+                            "kernel": f"fa_decode_kernel<{'bf16' if esz == 2 else 'f32'},{w.d},{1 if w.nq == 1 else 4}>"}
+        line["clocks"] = clocks.summary()
+        line["gpu_launches"] = a.steps
+    if "e2e" in legs:
+        # one generation step through the public API: the new tokens' q, k, v
+        # rows come from pinned host memory (k, v appended to the resident
+        # cache), o and lse go back to pinned host memory
+        q_h = q.cpu().pin_memory()
+        kn_h = k[:, :, w.nk - w.nq:].cpu().pin_memory()
+        vn_h = v[:, :, w.nk - w.nq:].cpu().pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(q_h, non_blocking=True)
+            k[:, :, w.nk - w.nq:].copy_(kn_h, non_blocking=True)
+            v[:, :, w.nk - w.nq:].copy_(vn_h, non_blocking=True)
+            step()
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+            stream.synchronize()
+
+        e2e_step()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fdist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(a.e2e_steps):
+            e2e_step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        fdist.barrier(dev)
+        e2e_ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.e2e_steps
+        line["e2e"] = {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": DECODE_UNIT, "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": 3 * q.numel() * esz,
+                       "d2h_bytes_per_step": o.numel() * esz + lse.numel() * 4,
+                       "api": "new q, k, v rows host->device, tiled_exact_attention_fa_b200.decode_into -> fa_decode "
+                              "(C ABI), o and lse device->host"}
+        if "value" not in line:
+            line["value"] = line["e2e"]["value"]
+    if "cpu" in legs and rank == 0 and world == 1:
+        import oracle
+        gbs, heads, dt = decode_cpu_sample(w, a.cpu_seconds, w.seed + 7)
+        line["cpu_baseline"] = {"value": gbs, "unit": DECODE_UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{heads} heads of {w.name} (fp64 oracle on host cores, {dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        fdist.barrier(dev)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     a = parse()
+    if a.path == "decode":
+        wd = W.DECODE_BY_NAME[a.decode_workload]
+        if a.impl == "reference":
+            return run_decode_reference(a, wd)
+        return run_decode(a, wd)
     w = W.BY_NAME[a.workload]
     if a.impl == "reference":
         return run_reference(a, w)

@@ -27,6 +27,7 @@
 #ifndef FA_B200_FA_H
 #define FA_B200_FA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -137,6 +138,46 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
 int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                 int64_t B, int64_t H, int64_t N, int64_t d,
                 float scale, int causal, int dtype, void* stream);
+
+/*
+ * fa_decode -- attention of Nq new queries over a key/value cache of Nk
+ * positions: the generation step ("FlashAttention: Tiled & Fused", card "KV
+ * Cache: Why Generation Speeds Up": past K and V are cached and each new
+ * token computes only its own).  The same operation as fa_fwd, with queries
+ * and keys of different lengths:
+ *
+ *   q        device, [B][H][Nq][d] of `dtype`: the new tokens' queries.
+ *   k, v     device, [B][H][Nk][d] of `dtype`: the cache, the new tokens'
+ *            own keys and values included as its last Nq rows.
+ *   o        device, [B][H][Nq][d] of `dtype`; lse device, [B][H][Nq] fp32
+ *            (natural log), each written once.
+ *   causal   0: every query uses all Nk keys; non-zero: query i sits at
+ *            position Nk - Nq + i and uses keys j <= Nk - Nq + i (needs
+ *            Nq <= Nk).  With Nq = 1 both are the same.
+ *   scale, dtype, stream: as for fa_fwd; d is 64 or 128.
+ *   workspace, workspace_bytes: device scratch of at least
+ *            fa_decode_workspace_bytes(B, H, Nq, Nk, d) bytes, 256-byte
+ *            aligned, no initialisation needed (the call clears the part it
+ *            uses as counters on `stream` first).  May be NULL when that size
+ *            is 0.  Calls that may run at the same time need separate
+ *            workspaces.
+ *
+ * The key range of each head is split into chunks that separate CTAs process
+ * (partial results merged by their log-sum-exp, as the online softmax
+ * merges tiles), so a single long head still uses the whole GPU.  Errors and
+ * asynchrony as for fa_fwd.  Alignment: q, k, v, o 16 bytes, lse 4 bytes.
+ */
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+              int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d,
+              float scale, int causal, int dtype,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_decode_workspace_bytes -- the workspace fa_decode needs for these sizes
+ * (0 when one CTA per head suffices, or for invalid sizes).  Depends only on
+ * the arguments, not on the device.
+ */
+size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d);
 
 /*
  * fa_check_device_status -- synchronise `stream`, then read and clear the

@@ -133,3 +133,38 @@ def test_host_entry_needs_no_alignment_but_a_gpu(lib):
     # host buffers need no alignment: a misaligned q passes the checks and the
     # call then fails on the missing GPU
     assert call_host(lib, q=A + 2) == fa.FA_ERR_CUDA
+
+
+def call_decode(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, Nq=1, Nk=128, d=128,
+                scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16, ws=A + 6 * NB, ws_bytes=1 << 20):
+    return lib.fa_decode(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(v=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nq=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nk=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nq=5, Nk=4, causal=1), fa.FA_ERR_INVALID_ARGUMENT),  # causal queries must fit in the cache
+    (dict(dtype=3), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(k=A + NB + 4), fa.FA_ERR_INVALID_ARGUMENT),         # misaligned
+    (dict(o=A + 64), fa.FA_ERR_INVALID_ARGUMENT),             # o overlaps q
+    (dict(Nk=1 << 20, ws=0), fa.FA_ERR_INVALID_ARGUMENT),     # a workspace is needed and missing
+    (dict(Nk=1 << 20, ws_bytes=16), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nk=1 << 20, ws=A + 6 * NB + 16), fa.FA_ERR_INVALID_ARGUMENT),  # workspace not 256-byte aligned
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+])
+def test_decode_rejected_before_cuda(lib, kwargs, code):
+    assert call_decode(lib, **kwargs) == code
+    assert lib.fa_last_error().decode() != ""
+
+
+def test_decode_workspace_size(lib):
+    # one CTA per head already fills the GPU: no workspace
+    assert lib.fa_decode_workspace_bytes(64, 32, 1, 4096, 128) == 0
+    # a single long head is split into chunks: partials (m, l, O) per chunk + counters
+    one = lib.fa_decode_workspace_bytes(1, 1, 1, 1 << 20, 128)
+    assert one > 0 and one % 256 == 0
+    assert lib.fa_decode_workspace_bytes(1, 1, 8, 1 << 20, 128) > one  # partials per query
+    assert lib.fa_decode_workspace_bytes(0, 1, 1, 10, 128) == 0       # invalid sizes

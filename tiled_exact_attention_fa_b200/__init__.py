@@ -36,6 +36,9 @@ _SIGNATURES = {
                        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                     [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "fa_decode": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 5 +
+                  [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "fa_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 5),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
@@ -162,6 +165,70 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float |
         out[0].copy_(o)
         out[1].copy_(lse)
         return out
+    return o, lse
+
+
+_decode_workspace: dict[int, torch.Tensor] = {}
+
+
+def decode_workspace(B: int, H: int, Nq: int, Nk: int, d: int, device=None) -> torch.Tensor | None:
+    """A device workspace large enough for fa_decode at these sizes, cached
+    per device and grown when needed (None when none is needed)."""
+    need = int(library().fa_decode_workspace_bytes(B, H, Nq, Nk, d))
+    if need == 0:
+        return None
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _decode_workspace.get(idx)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
+        _decode_workspace[idx] = ws
+    return ws
+
+
+def decode_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor, *,
+                scale: float | None = None, causal: bool = False, workspace: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None) -> None:
+    """fa_decode into caller-provided CUDA tensors: q, o [B,H,Nq,d], k, v
+    [B,H,Nk,d] (the cache), lse [B,H,Nq] fp32.  `workspace` defaults to a
+    per-device cached one, so calls that may overlap on the GPU (different
+    streams) must pass their own."""
+    if q.dtype not in _DTYPES or not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise TypeError("q, k, v, o must all be bf16 or all fp32")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be fp32")
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape or o.shape != q.shape:
+        raise ValueError("q, o must be [B, H, Nq, d] and k, v [B, H, Nk, d]")
+    if q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3] or lse.shape != q.shape[:3]:
+        raise ValueError("inconsistent shapes")
+    for t in (q, k, v, o, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("decode_into needs contiguous CUDA tensors")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            workspace = decode_workspace(B, H, Nq, Nk, d, q.device)
+        ptr, size = (0, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        if ptr % 256:
+            off = 256 - ptr % 256
+            ptr, size = ptr + off, size - off
+        s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+        _check(int(library().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                       B, H, Nq, Nk, d, float(scale), int(causal), _DTYPES[q.dtype],
+                                       ptr or None, size, s)))
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
+           causal: bool = False):
+    """Attention of the new queries q [B,H,Nq,d] over the cache k, v
+    [B,H,Nk,d] (CUDA tensors).  Returns (o, lse)."""
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    decode_into(q, k, v, o, lse, scale=scale, causal=causal)
     return o, lse
 
 

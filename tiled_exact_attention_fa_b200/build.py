@@ -49,18 +49,29 @@ def _inputs_digest() -> str:
 _TOKENS = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'', re.S)
 
 
-def code_digest() -> str:
-    """Digest of the library's code with comments and layout removed: it
-    changes when the compiled code can change, not when a comment does."""
+def code_digest(files=None) -> str:
+    """Digest of the library's code (or of the given csrc files) with comments
+    and layout removed: it changes when the compiled code can change, not
+    when a comment does."""
     h = hashlib.sha1()
-    for d in (CSRC, INCLUDE):
-        for name in sorted(os.listdir(d)):
-            if name.endswith((".cu", ".cuh", ".h")):
-                with open(os.path.join(d, name)) as f:
-                    text = _TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), f.read())
-                h.update(name.encode() + " ".join(text.split()).encode())
+    if files is None:
+        paths = [os.path.join(d, n) for d in (CSRC, INCLUDE) for n in sorted(os.listdir(d))
+                 if n.endswith((".cu", ".cuh", ".h"))]
+    else:
+        paths = [os.path.join(CSRC, n) for n in files]
+    for path in paths:
+        with open(path) as f:
+            text = _TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), f.read())
+        h.update(os.path.basename(path).encode() + " ".join(text.split()).encode())
     h.update(" ".join(ARCH + FLAGS).encode())
     return h.hexdigest()
+
+
+# the sources each kernel is compiled from (for records tied to one kernel)
+KERNEL_SOURCES = {
+    "forward": ["fa_fwd_tc.cuh", "sm100_ptx.cuh"],
+    "decode": ["fa_decode.cuh", "sm100_ptx.cuh"],
+}
 
 
 def is_current() -> bool:

@@ -16,6 +16,7 @@
 
 #include "fa.h"
 #include "fa_testing.h"
+#include "fa_decode.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 
@@ -53,6 +54,7 @@ struct DeviceState {
     int sm_count = 0;
     int cc_major = 0;
     bool smem_raised[4] = {false, false, false, false};
+    bool decode_smem_raised[8] = {false, false, false, false, false, false, false, false};
 };
 
 constexpr int kMaxDevices = 64;
@@ -586,4 +588,143 @@ extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o,
     // the caller's stream continues once the last copy-out is done
     if ((rc = ck(cudaEventRecord(pp.ev_done, pp.s_out), "cudaEventRecord")) != FA_OK) return rc;
     return ck(cudaStreamWaitEvent(caller, pp.ev_done, 0), "cudaStreamWaitEvent");
+}
+
+// ---------------------------------------------------------------------------
+// fa_decode: a few new queries over a key/value cache (split-KV, see
+// fa_decode.cuh).  The chunking depends only on the arguments, so the
+// workspace size can be computed before the call.
+namespace {
+
+constexpr int64_t kDecodeTargetCtas = 1184;  // 148 SMs x 8: the grid covers a B200 several times
+constexpr int64_t kDecodeMinChunk = 256;     // keys; below this a CTA's fixed costs dominate
+
+struct DecodePlan {
+    int64_t bh = 0, groups = 0, chunks = 0, chunk = 0, nq_tile = 0;
+    size_t part_bytes = 0, count_bytes = 0, workspace = 0;
+};
+
+DecodePlan decode_plan(int64_t bh, int64_t nq, int64_t nk, int64_t d) {
+    DecodePlan pl;
+    pl.bh = bh;
+    pl.nq_tile = nq == 1 ? 1 : fa::dec::kMaxQ;
+    pl.groups = (nq + pl.nq_tile - 1) / pl.nq_tile;
+    const int64_t ctas = bh * pl.groups;
+    int64_t chunks = (kDecodeTargetCtas + ctas - 1) / ctas;
+    const int64_t max_chunks = (nk + kDecodeMinChunk - 1) / kDecodeMinChunk;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    int64_t chunk = (nk + chunks - 1) / chunks;
+    chunk = (chunk + fa::dec::kTileKeys - 1) / fa::dec::kTileKeys * fa::dec::kTileKeys;
+    pl.chunk = chunk;
+    pl.chunks = (nk + chunk - 1) / chunk;
+    if (pl.chunks > 1) {
+        pl.part_bytes = round_up(static_cast<size_t>(bh * nq * pl.chunks * (d + 2)) * 4, 256);
+        pl.count_bytes = round_up(static_cast<size_t>(bh * pl.groups) * 4, 256);
+    }
+    pl.workspace = pl.part_bytes + pl.count_bytes;
+    return pl;
+}
+
+int decode_check(const void* q, const void* k, const void* v, const void* o, const float* lse, int64_t B,
+                 int64_t H, int64_t Nq, int64_t Nk, int64_t d, float scale, int causal, int dtype, DecodePlan* pl) {
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1)
+        return fail(FA_ERR_INVALID_ARGUMENT, "B, H, Nq, Nk and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (causal && Nq > Nk) return fail(FA_ERR_INVALID_ARGUMENT, "causal needs Nq <= Nk (the queries are the last Nq positions)");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (Nk > (int64_t{1} << 30) || Nq > (int64_t{1} << 20)) return fail(FA_ERR_INVALID_ARGUMENT, "Nk or Nq too large");
+    if (B > (int64_t{1} << 24) / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    const int64_t bh = B * H;
+    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
+    *pl = decode_plan(bh, Nq, Nk, d);
+    if (pl->groups > 65535) return fail(FA_ERR_INVALID_ARGUMENT, "too many query groups");
+    if (bh * pl->chunks > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * chunks too large");
+    auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16))
+        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+    if (misaligned(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    const size_t qb = static_cast<size_t>(bh * Nq * d * elem), kb = static_cast<size_t>(bh * Nk * d * elem);
+    const size_t lb = static_cast<size_t>(bh * Nq * 4);
+    if (overlaps(o, qb, q, qb) || overlaps(o, qb, k, kb) || overlaps(o, qb, v, kb) || overlaps(o, qb, lse, lb))
+        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
+    if (overlaps(lse, lb, q, qb) || overlaps(lse, lb, k, kb) || overlaps(lse, lb, v, kb))
+        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
+    return FA_OK;
+}
+
+template <typename T, int D, int NQ>
+int launch_decode(DeviceState* st, int slot, const fa::dec::Params& p, const DecodePlan& pl, cudaStream_t s) {
+    using C = fa::dec::Cfg<T, D>;
+    auto kernel = fa::dec::fa_decode_kernel<T, D, NQ>;
+    if (!st->decode_smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->decode_smem_raised[slot] = true;
+    }
+    dim3 grid(static_cast<unsigned>(pl.bh * pl.chunks), static_cast<unsigned>(pl.groups));
+    kernel<<<grid, fa::dec::kThreads, C::kSmemBytes, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the decode kernel");
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d) {
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || B > (int64_t{1} << 24) / H) return 0;
+    return decode_plan(B * H, Nq, Nk, d).workspace;
+}
+
+extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                         int64_t Nq, int64_t Nk, int64_t d, float scale, int causal, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    g_last_error.clear();
+    DecodePlan pl;
+    int rc = decode_check(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, &pl);
+    if (rc != FA_OK) return rc;
+    if (pl.workspace > 0) {
+        if (!workspace || workspace_bytes < pl.workspace)
+            return fail(FA_ERR_INVALID_ARGUMENT, "workspace missing or smaller than fa_decode_workspace_bytes()");
+        if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+            return fail(FA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
+    }
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    fa::dec::Params p;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.lse = lse;
+    p.part = pl.workspace ? static_cast<float*>(workspace) : nullptr;
+    p.count = pl.workspace ? reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.part_bytes) : nullptr;
+    p.status = st->status;
+    p.nq = static_cast<int>(Nq);
+    p.nk = static_cast<int>(Nk);
+    p.chunk = static_cast<int>(pl.chunk);
+    p.chunks = static_cast<int>(pl.chunks);
+    p.groups = static_cast<int>(pl.groups);
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.causal = causal != 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the chunk counters start from zero on every call (the workspace may
+    // have held other sizes' partials since)
+    if (pl.workspace > 0) {
+        cudaError_t e = cudaMemsetAsync(p.count, 0, pl.count_bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode counters)");
+    }
+    const bool one = pl.nq_tile == 1;
+    if (dtype == FA_DTYPE_BF16) {
+        if (d == 128) return one ? launch_decode<__nv_bfloat16, 128, 1>(st, 0, p, pl, s)
+                                 : launch_decode<__nv_bfloat16, 128, fa::dec::kMaxQ>(st, 1, p, pl, s);
+        return one ? launch_decode<__nv_bfloat16, 64, 1>(st, 2, p, pl, s)
+                   : launch_decode<__nv_bfloat16, 64, fa::dec::kMaxQ>(st, 3, p, pl, s);
+    }
+    if (d == 128) return one ? launch_decode<float, 128, 1>(st, 4, p, pl, s)
+                             : launch_decode<float, 128, fa::dec::kMaxQ>(st, 5, p, pl, s);
+    return one ? launch_decode<float, 64, 1>(st, 6, p, pl, s) : launch_decode<float, 64, fa::dec::kMaxQ>(st, 7, p, pl, s);
 }

@@ -109,3 +109,56 @@ def sample_rows(w: Workload, per_head: int | None = None):
                     seen.add(r)
             out[b, h] = torch.tensor(sorted(chosen), dtype=torch.int64)
     return out
+
+
+# ------------------------------------------------------------------ decode
+# A generation step over a key/value cache ("FlashAttention: Tiled & Fused",
+# card "KV Cache: Why Generation Speeds Up"): nq new queries per head over a
+# cache of nk positions whose last nq rows are the new tokens' own keys and
+# values.  Same recipe: iid standard normal, drawn Q, K, V in that order.
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    dtype: torch.dtype
+    B: int
+    H: int
+    nq: int
+    nk: int
+    d: int
+    causal: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def cache_bytes(self) -> int:
+        """K and V of the cache: what one step must read from HBM."""
+        return 2 * self.B * self.H * self.nk * self.d * (2 if self.dtype == torch.bfloat16 else 4)
+
+
+DECODE_WORKLOADS = [
+    # a batch of 16 sequences of 16k cached tokens, 32 heads: 4.3 GB of cache per step
+    DecodeWorkload("bf16_decode_b16h32_q1_nk16384_d128", torch.bfloat16, 16, 32, 1, 16384, 128, True, 5),
+    # one long sequence, 8 heads, 256k cached tokens: split-KV over ~150 chunks per head
+    DecodeWorkload("bf16_decode_b1h8_q1_nk262144_d128", torch.bfloat16, 1, 8, 1, 262144, 128, True, 6),
+    # four new tokens at once (speculative / chunked step), causal among them
+    DecodeWorkload("bf16_decode_b8h32_q4_nk32768_d128", torch.bfloat16, 8, 32, 4, 32768, 128, True, 7),
+]
+DECODE_BY_NAME = {w.name: w for w in DECODE_WORKLOADS}
+DECODE_HEADLINE = DECODE_BY_NAME["bf16_decode_b16h32_q1_nk16384_d128"]
+
+
+def make_decode_inputs(w: DecodeWorkload, device: str | torch.device = "cpu", pin: bool = False):
+    """q [B,H,nq,d], k, v [B,H,nk,d] for decode workload ``w`` (seeded, CPU-drawn:
+    Q, then K, then V, each as B consecutive draws of one batch element's
+    [H, n, d] in fp32, cast to the workload's dtype)."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    out = []
+    for n in (w.nq, w.nk, w.nk):
+        x = torch.empty((w.B, w.H, n, w.d), dtype=w.dtype, pin_memory=pin)
+        for b in range(w.B):
+            x[b] = torch.randn((w.H, n, w.d), generator=g, dtype=torch.float32).to(w.dtype)
+        out.append(x.to(device) if str(device) != "cpu" else x)
+    return tuple(out)
