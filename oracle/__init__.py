@@ -69,6 +69,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     g.restype = ctypes.c_int
     g.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 4 + [
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    b = lib.oracle_attention_bwd
+    b.restype = ctypes.c_int
+    b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_version.restype = ctypes.c_int
     return lib
@@ -144,3 +148,20 @@ def attention_decode(q, k, v, scale: float, causal: bool, lib=None):
     if rc != 0:
         raise RuntimeError(f"oracle_attention_decode failed with code {rc}")
     return o, lse
+
+
+def attention_bwd(q, k, v, do, scale: float, causal: bool, lib=None):
+    """Gradients (dq, dk, dv) of the attention output with respect to q, k, v
+    for the upstream gradient `do`, in fp64.  All inputs [B, H, N, d] (exact
+    values, fp32); returns three [B, H, N, d] fp64 arrays."""
+    lib = lib or load()
+    q, k, v, do = (np.ascontiguousarray(x, dtype=np.float32) for x in (q, k, v, do))
+    if q.ndim != 4 or not (q.shape == k.shape == v.shape == do.shape):
+        raise ValueError("q, k, v, do must share one [B, H, N, d] shape")
+    B, H, N, d = q.shape
+    dq, dk, dv = (np.empty((B, H, N, d), dtype=np.float64) for _ in range(3))
+    rc = lib.oracle_attention_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, do.ctypes.data, B * H, N, d,
+                                  float(scale), int(bool(causal)), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_bwd failed with code {rc}")
+    return dq, dk, dv

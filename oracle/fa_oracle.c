@@ -216,3 +216,111 @@ int oracle_attention_decode(const float* q, const float* k, const float* v,
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * oracle_attention_bwd -- gradients of the same attention with respect to
+ * Q, K and V for an upstream gradient dO of the output.  The pages give the
+ * forward only and name training as what the method enables ("FlashAttention:
+ * Tiled & Fused", section "Enabling longer contexts in training and
+ * inference"); the plain reading is the gradient of the exact function,
+ * written out from its definition with every score matrix materialised:
+ *
+ *     P  = softmax(scale * Q K^T [causal])          (two passes per row)
+ *     dV = P^T dO
+ *     dP = dO V^T
+ *     dS = P * (dP - rowsum(dO * O)),  O = P V       (softmax Jacobian)
+ *     dQ = scale * dS K,   dK = scale * dS^T Q
+ *
+ *   q, k, v, dout: [bh][n][d] fp32        dq, dk, dv: [bh][n][d] fp64
+ * Memory: three n x n fp64 matrices per head at a time.
+ * Returns 0 on success, -1 on bad arguments, -2 if scratch cannot be allocated.
+ */
+int oracle_attention_bwd(const float* q, const float* k, const float* v, const float* dout,
+                         int64_t bh, int64_t n, int64_t d, double scale, int causal,
+                         double* dq, double* dk, double* dv) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    if (bh <= 0 || n <= 0 || d <= 0) return -1;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t h = 0; h < bh; ++h) {
+        double* pm = (double*)malloc((size_t)(n * n) * sizeof(double));   /* P */
+        double* gm = (double*)malloc((size_t)(n * n) * sizeof(double));   /* dP, then dS */
+        double* om = (double*)malloc((size_t)(n * d) * sizeof(double));   /* O */
+        if (!pm || !gm || !om) {
+#pragma omp atomic write
+            failed = 1;
+            free(pm);
+            free(gm);
+            free(om);
+            continue;
+        }
+        const float* qh = q + h * n * d;
+        const float* kh = k + h * n * d;
+        const float* vh = v + h * n * d;
+        const float* gh = dout + h * n * d;
+        /* P, row by row */
+        for (int64_t r = 0; r < n; ++r) {
+            double* prow = pm + r * n;
+            double mrow = -INFINITY;
+            for (int64_t c = 0; c < n; ++c) {
+                if (causal && c > r) {
+                    prow[c] = -INFINITY;
+                    continue;
+                }
+                double acc = 0.0;
+                for (int64_t t = 0; t < d; ++t) acc += (double)qh[r * d + t] * (double)kh[c * d + t];
+                prow[c] = scale * acc;
+                if (prow[c] > mrow) mrow = prow[c];
+            }
+            double tot = 0.0;
+            for (int64_t c = 0; c < n; ++c) {
+                prow[c] = exp(prow[c] - mrow);
+                tot += prow[c];
+            }
+            for (int64_t c = 0; c < n; ++c) prow[c] /= tot;
+        }
+        /* O = P V and dP = dO V^T */
+        for (int64_t r = 0; r < n; ++r)
+            for (int64_t t = 0; t < d; ++t) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < n; ++c) acc += pm[r * n + c] * (double)vh[c * d + t];
+                om[r * d + t] = acc;
+            }
+        for (int64_t r = 0; r < n; ++r)
+            for (int64_t c = 0; c < n; ++c) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)vh[c * d + t];
+                gm[r * n + c] = acc;
+            }
+        /* dS = P * (dP - rowsum(dO * O)) */
+        for (int64_t r = 0; r < n; ++r) {
+            double drow = 0.0;
+            for (int64_t t = 0; t < d; ++t) drow += (double)gh[r * d + t] * om[r * d + t];
+            for (int64_t c = 0; c < n; ++c) gm[r * n + c] = pm[r * n + c] * (gm[r * n + c] - drow);
+        }
+        /* dV = P^T dO, dK = scale dS^T Q, dQ = scale dS K */
+        double* dvh = dv + h * n * d;
+        double* dkh = dk + h * n * d;
+        double* dqh = dq + h * n * d;
+        for (int64_t c = 0; c < n; ++c)
+            for (int64_t t = 0; t < d; ++t) {
+                double av = 0.0, ak = 0.0;
+                for (int64_t r = 0; r < n; ++r) {
+                    av += pm[r * n + c] * (double)gh[r * d + t];
+                    ak += gm[r * n + c] * (double)qh[r * d + t];
+                }
+                dvh[c * d + t] = av;
+                dkh[c * d + t] = scale * ak;
+            }
+        for (int64_t r = 0; r < n; ++r)
+            for (int64_t t = 0; t < d; ++t) {
+                double aq = 0.0;
+                for (int64_t c = 0; c < n; ++c) aq += gm[r * n + c] * (double)kh[c * d + t];
+                dqh[r * d + t] = scale * aq;
+            }
+        free(pm);
+        free(gm);
+        free(om);
+    }
+    return failed ? -2 : 0;
+}

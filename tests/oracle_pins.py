@@ -368,6 +368,77 @@ def pin_decode_torch_sdpa(lib):
         np.testing.assert_allclose(lse, lse_ref.numpy(), rtol=0, atol=1e-12)
 
 
+# --------------------------------------------------------------- backward pass
+# The gradient of the exact function (the pages name training as what the
+# method enables; they give no backward formulas).
+
+def _bwd(lib, q, k, v, do, scale, causal):
+    return oracle.attention_bwd(q, k, v, do, scale, causal, lib=lib)
+
+
+def pin_bwd_torch_autograd(lib):
+    """torch's fp64 autograd through its math attention (explicit scale)."""
+    for (B, H, N, d, causal, seed) in [(1, 2, 33, 8, False, 80), (2, 1, 70, 16, True, 81)]:
+        q, k, v, do = (_rand((B, H, N, d), seed + i) for i in range(4))
+        dq, dk, dv = _bwd(lib, q, k, v, do, 0.35, causal)
+        tq, tk, tv = (torch.from_numpy(x.astype(np.float64)).requires_grad_() for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=0.35)
+        o.backward(torch.from_numpy(do.astype(np.float64)))
+        for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-12)
+
+
+def pin_bwd_finite_differences(lib):
+    """Central differences of L = sum(O * dO), computed with the forward
+    oracle, against the gradients at a few entries of q, k and v."""
+    B, H, N, d = 1, 1, 6, 3
+    q, k, v, do = (_rand((B, H, N, d), 90 + i) for i in range(4))
+    for causal in (False, True):
+        dq, dk, dv = _bwd(lib, q, k, v, do, 0.8, causal)
+
+        def loss(qq, kk, vv):
+            o, _ = _run(lib, qq, kk, vv, 0.8, causal)
+            return float((o * do.astype(np.float64)).sum())
+
+        h = 2.0 ** -10  # float32 inputs: steps of 2^-10 are exact, the loss is smooth
+        for (which, grad) in ((0, dq), (1, dk), (2, dv)):
+            for (i, t) in ((0, 0), (3, 2), (5, 1)):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][0, 0, i, t] += h
+                up = loss(*args)
+                args[which][0, 0, i, t] -= 2 * h
+                dn = loss(*args)
+                fd = (up - dn) / (2 * h)
+                assert abs(fd - grad[0, 0, i, t]) < 2e-5, (which, i, t, fd, grad[0, 0, i, t])
+
+
+def pin_bwd_invariants(lib):
+    """Rows of dS sum to zero, so the key gradients of a head sum to zero and
+    constant keys give no query gradient; rows of P sum to one, so the value
+    gradients of a head sum to the sum of dO; the gradients are linear in dO
+    and vanish with it."""
+    B, H, N, d = 1, 2, 29, 8
+    q, k, v, do, do2 = (_rand((B, H, N, d), 100 + i) for i in range(5))
+    # upstream gradients on a 2^-8 grid, so that 2 do - 3 do2 is exact in fp32
+    do, do2 = (np.round(x * 256.0).astype(np.float32) / np.float32(256.0) for x in (do, do2))
+    for causal in (False, True):
+        dq, dk, dv = _bwd(lib, q, k, v, do, 0.5, causal)
+        np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+        np.testing.assert_allclose(dv.sum(axis=2), do.astype(np.float64).sum(axis=2), atol=1e-12)
+        kc = np.broadcast_to(k[:, :, :1], k.shape).copy()
+        dqc, _, _ = _bwd(lib, q, kc, v, do, 0.5, causal)
+        np.testing.assert_allclose(dqc, 0.0, atol=1e-12)
+        z = _bwd(lib, q, k, v, np.zeros_like(do), 0.5, causal)
+        for g in z:
+            assert np.abs(g).max() == 0.0
+        g1 = _bwd(lib, q, k, v, do2, 0.5, causal)
+        gs = _bwd(lib, q, k, v, (2 * do - 3 * do2).astype(np.float32), 0.5, causal)
+        for a, b, c in zip((dq, dk, dv), g1, gs):
+            np.testing.assert_allclose(c, 2 * a - 3 * b, atol=1e-11)
+
+
+BWD_PINS = [pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants]
+
 DECODE_PINS = [pin_decode_hand_worked, pin_decode_closed_forms, pin_decode_is_the_last_rows_of_prefill,
                pin_decode_future_keys_ignored, pin_decode_torch_sdpa]
 
@@ -375,4 +446,4 @@ ALL_PINS = [
     pin_hand_worked, pin_q_zero_mean_of_v, pin_single_key, pin_causal_row0, pin_affine_v,
     pin_key_permutation, pin_future_keys_ignored, pin_softmax_shift, pin_lse_bounds,
     pin_row_subset, pin_online_ledger, pin_torch_sdpa,
-] + DECODE_PINS
+] + DECODE_PINS + BWD_PINS

@@ -39,6 +39,18 @@ MUTANTS = [
     ("decode_not_normalised", "orow[t] = acc / sum;", "orow[t] = acc;"),
     ("decode_v_of_key_0", "acc += w[kj] * (double)vh[kj * d + t];", "acc += w[kj] * (double)vh[t];"),
     ("decode_query_of_head_0", "const float* qrow = q + (h * nq + qi) * d;", "const float* qrow = q + qi * d;"),
+    # the backward pass
+    ("bwd_dk_scale_dropped", "dkh[c * d + t] = scale * ak;", "dkh[c * d + t] = ak;"),
+    ("bwd_dq_scale_dropped", "dqh[r * d + t] = scale * aq;", "dqh[r * d + t] = aq;"),
+    ("bwd_no_softmax_jacobian", "gm[r * n + c] = pm[r * n + c] * (gm[r * n + c] - drow);",
+     "gm[r * n + c] = pm[r * n + c] * gm[r * n + c];"),
+    ("bwd_ds_without_p", "gm[r * n + c] = pm[r * n + c] * (gm[r * n + c] - drow);",
+     "gm[r * n + c] = gm[r * n + c] - drow;"),
+    ("bwd_dv_from_p_not_transposed", "av += pm[r * n + c] * (double)gh[r * d + t];",
+     "av += pm[c * n + r] * (double)gh[r * d + t];"),
+    ("bwd_mask_off", "if (causal && c > r) {", "if (0 && causal && c > r) {"),
+    ("bwd_dp_with_k", "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)vh[c * d + t];",
+     "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)kh[c * d + t];"),
 ]
 
 
