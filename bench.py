@@ -15,7 +15,9 @@ slowest rank's.
 `--impl reference` times the fp64 CPU oracle (test infrastructure, the
 deliberately slow plain definition) on a bounded sample of the same workload.
 
-`--path decode` measures the generation step instead (fa_decode: new queries
+`--path backward` measures fa_bwd (dq, dk, dv from the saved lse) on the same
+workload, counting the customary 2.5x the forward's FLOPs.  `--path decode`
+measures the generation step instead (fa_decode: new queries
 over a resident key/value cache, HBM-bound): the metric is the cache bytes
 read per second, against the measured HBM copy bandwidth.
 """
@@ -57,7 +59,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
-    ap.add_argument("--path", default="forward", choices=["forward", "decode"])
+    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward"])
     ap.add_argument("--decode-workload", default=W.DECODE_HEADLINE.name, choices=sorted(W.DECODE_BY_NAME))
     return ap.parse_args()
 
@@ -486,8 +488,139 @@ def run_decode(a, w: W.DecodeWorkload):
     return 0
 
 
+BWD_METRIC = "attention bwd TFLOPS (bf16, d=128, N=8K causal; 10*B*H*N^2*d, halved for causal) and % of B200 dense BF16 peak"
+
+
+def bwd_cpu_sample(w: W.Workload, seconds: float, seed: int):
+    """fp64 oracle backward on whole heads of a shorter sequence (N = 512) of
+    the workload's shape; returns (TFLOP/s in the metric's count, heads, s)."""
+    import oracle
+    n = min(w.N, 512)
+    g = torch.Generator().manual_seed(seed)
+
+    def run(heads):
+        x = [torch.randn((1, heads, n, w.d), generator=g).to(w.dtype).float().numpy() for _ in range(4)]
+        t0 = time.perf_counter()
+        oracle.attention_bwd(*x, w.scale, w.causal)
+        return time.perf_counter() - t0
+
+    dt = run(1)
+    heads = int(max(1, min(w.B * w.H, oracle.num_threads() * max(1, int(seconds / max(dt, 1e-6))))))
+    dt = run(heads)
+    flops = 2.5 * accounting.attention_flops(1, heads, n, w.d, w.causal)
+    return flops / dt / 1e12, heads, dt, n
+
+
+def run_backward(a, w: W.Workload):
+    import tiled_exact_attention_fa_b200 as fa
+
+    rank, local_rank, world = fdist.env_world()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        fdist.init("nccl", timeout_s=300)
+    legs = set(a.legs.split(","))
+    wr = W.Workload(w.name, w.dtype, w.B, w.H, w.N, w.d, w.causal, w.seed + 1000 * rank, w.q_mult)
+    q_h, k_h, v_h = W.make_inputs(wr, pin=True)
+    g = torch.Generator().manual_seed(wr.seed + 500)
+    do_h = torch.randn(q_h.shape, generator=g).to(w.dtype).pin_memory()
+    q, k, v, do = (x.to(dev, non_blocking=True) for x in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    fa.forward_into(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(int(fa.library().fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = 2.5 * accounting.attention_flops(w.B, w.H, w.N, w.d, w.causal)
+
+    def step():
+        fa.backward_into(q, k, v, o, lse, do, dq, dk, dv, scale=w.scale, causal=w.causal, workspace=ws)
+
+    for _ in range(a.warmup):
+        step()
+    fa.check_device_status()
+    line = {"metric": BWD_METRIC, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                       "seed": w.seed, "pass": "backward (dq, dk, dv from the saved lse)",
+                       "per_rank": "own seeded batch (seed + 1000*rank), no collective",
+                       "l2": "inputs > L2, no flush", "flop_per_step": flops,
+                       "mma_flop_per_step": 1.4 * flops}}
+    if "kernel" in legs:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
+            fdist.barrier(dev)
+            torch.cuda.synchronize(dev)
+            start.record(stream)
+            for _ in range(a.steps):
+                step()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+            fdist.barrier(dev)
+        fa.check_device_status()
+        ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.steps
+        tf = flops / (ms * 1e-3) / 1e12
+        peak, peak_sus, _, peak_kind = measured_peaks()
+        line["value"] = world * tf
+        line["ms_per_step"] = ms
+        line["pct_of_bf16_peak"] = 100.0 * tf / peak
+        line["roofline"] = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                            "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)", "frac_of_sustained": tf / peak_sus,
+                            "traffic": None, "kernel": "fa_bwd_dq_kernel + fa_bwd_dkdv_kernel (+ row-dot)",
+                            "note": "achieved counts 10*N^2*d; the kernels recompute S and dP (14*N^2*d on the tensor cores)"}
+        line["clocks"] = clocks.summary()
+        line["gpu_launches"] = 3 * a.steps
+    if "e2e" in legs:
+        o_h = o.cpu().pin_memory()
+        lse_h = lse.cpu().pin_memory()
+        outs = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3)]
+
+        def e2e_step():
+            for dst, src in ((q, q_h), (k, k_h), (v, v_h), (o, o_h), (lse, lse_h), (do, do_h)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(outs, (dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+            stream.synchronize()
+
+        e2e_step()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fdist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(a.e2e_steps):
+            e2e_step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        fdist.barrier(dev)
+        e2e_ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.e2e_steps
+        tb = q.numel() * q.element_size()
+        line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": 5 * tb + lse.numel() * 4, "d2h_bytes_per_step": 3 * tb,
+                       "api": "host tensors -> device, tiled_exact_attention_fa_b200.backward_into -> fa_bwd, "
+                              "dq, dk, dv -> host"}
+        if "value" not in line:
+            line["value"] = line["e2e"]["value"]
+    if "cpu" in legs and rank == 0 and world == 1:
+        import oracle
+        tf, heads, dt, n = bwd_cpu_sample(w, a.cpu_seconds, w.seed + 7)
+        line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{heads} heads of N={n} (d={w.d}, causal={w.causal}) through the fp64 "
+                                          f"backward oracle, {dt:.1f} s; work counted as the metric counts it"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        fdist.barrier(dev)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     a = parse()
+    if a.path == "backward":
+        return run_backward(a, W.BY_NAME[a.workload])
     if a.path == "decode":
         wd = W.DECODE_BY_NAME[a.decode_workload]
         if a.impl == "reference":

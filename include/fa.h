@@ -180,6 +180,36 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
 size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d);
 
 /*
+ * fa_bwd -- gradients of fa_fwd: given the forward's q, k, v, o and lse and
+ * the gradient dout of a loss with respect to o, writes dq, dk, dv (the
+ * gradient of the exact function; the pages give the forward only and name
+ * training as what the method enables -- "FlashAttention: Tiled & Fused",
+ * "Enabling longer contexts in training and inference"):
+ *
+ *   P = exp(scale * q k^T - lse) [causal],  D = rowsum(dout * o)
+ *   dv = P^T dout,  dS = P * (dout v^T - D),  dq = scale dS k,  dk = scale dS^T q
+ *
+ *   q, k, v, o, dout  device, [B][H][N][d] bf16 (o and lse exactly as fa_fwd
+ *                     wrote them); lse device [B][H][N] fp32.
+ *   dq, dk, dv        device, [B][H][N][d] bf16, written once.
+ *   workspace         device scratch of fa_bwd_workspace_bytes(B, H, N, d)
+ *                     bytes (D for every row), 16-byte aligned.
+ *   scale, causal     as for fa_fwd; dtype must be FA_DTYPE_BF16
+ *                     (FA_ERR_UNSUPPORTED otherwise); d is 64 or 128.
+ * No score matrix reaches memory: P is recomputed tile by tile from lse.
+ * Asynchronous on `stream` (three kernel launches); argument errors are
+ * reported before any CUDA call.  Alignment 16 bytes (lse 4).  Outputs and
+ * workspace must not overlap the inputs or each other.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv,
+           int64_t B, int64_t H, int64_t N, int64_t d, float scale, int causal, int dtype,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/* fa_bwd_workspace_bytes -- the workspace fa_bwd needs (0 for invalid sizes). */
+size_t fa_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
  * fa_check_device_status -- synchronise `stream`, then read and clear the
  * library's device status word for the current device.  Returns FA_OK,
  * FA_ERR_DEVICE_TIMEOUT when a kernel launched by this library gave up on a

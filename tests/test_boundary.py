@@ -168,3 +168,22 @@ def test_decode_workspace_size(lib):
     assert one > 0 and one % 256 == 0
     assert lib.fa_decode_workspace_bytes(1, 1, 8, 1 << 20, 128) > one  # partials per query
     assert lib.fa_decode_workspace_bytes(0, 1, 1, 10, 128) == 0       # invalid sizes
+
+
+def test_backward_rejected_before_cuda(lib):
+    args = [A, A + NB, A + 2 * NB, A + 3 * NB, A + 4 * NB, A + 5 * NB, A + 6 * NB, A + 7 * NB, A + 8 * NB]
+    ok = dict(B=1, H=1, N=128, d=128, scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16, ws=A + 9 * NB, wsb=1 << 20)
+
+    def bwd(args, B=1, H=1, N=128, d=128, scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16, ws=A + 9 * NB, wsb=1 << 20):
+        return lib.fa_bwd(*args, B, H, N, d, scale, causal, dtype, ws, wsb, None)
+
+    assert bwd([0] + args[1:]) == fa.FA_ERR_INVALID_ARGUMENT          # null q
+    assert bwd(args, N=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert bwd(args, dtype=fa.FA_DTYPE_F32) == fa.FA_ERR_UNSUPPORTED   # bf16 only
+    assert bwd(args, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert bwd(args, ws=0) == fa.FA_ERR_INVALID_ARGUMENT               # workspace missing
+    assert bwd(args, wsb=4) == fa.FA_ERR_INVALID_ARGUMENT              # workspace too small
+    assert bwd(args[:6] + [A + 16] + args[7:]) == fa.FA_ERR_INVALID_ARGUMENT  # dq overlaps q
+    assert bwd(args[:6] + [A + 6 * NB + 8] + args[7:]) == fa.FA_ERR_INVALID_ARGUMENT  # misaligned
+    assert lib.fa_bwd_workspace_bytes(2, 3, 1000, 128) >= 2 * 3 * 1000 * 4
+    assert lib.fa_bwd_workspace_bytes(0, 3, 1000, 128) == 0

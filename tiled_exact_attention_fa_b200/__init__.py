@@ -39,6 +39,9 @@ _SIGNATURES = {
     "fa_decode": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 5 +
                   [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fa_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 5),
+    "fa_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int64] * 4 +
+               [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "fa_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 4),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
@@ -230,6 +233,40 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | 
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     decode_into(q, k, v, o, lse, scale=scale, causal=causal)
     return o, lse
+
+
+def backward_into(q, k, v, o, lse, dout, dq, dk, dv, *, scale: float | None = None, causal: bool = False,
+                  workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> None:
+    """fa_bwd into caller-provided CUDA tensors (all [B, H, N, d] bf16, lse
+    [B, H, N] fp32 as the forward wrote it)."""
+    ts = (q, k, v, o, dout, dq, dk, dv)
+    if any(t.dtype != torch.bfloat16 for t in ts) or lse.dtype != torch.float32:
+        raise TypeError("the backward takes bf16 tensors and an fp32 lse")
+    if any(t.shape != q.shape for t in ts) or q.dim() != 4 or lse.shape != q.shape[:3]:
+        raise ValueError("all tensors must be [B, H, N, d], lse [B, H, N]")
+    for t in ts + (lse,):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("backward_into needs contiguous CUDA tensors")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = int(library().fa_bwd_workspace_bytes(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+        _check(int(library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                    dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                                    float(scale), int(causal), FA_DTYPE_BF16, workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(), s)))
+
+
+def backward(q, k, v, o, lse, dout, *, scale: float | None = None, causal: bool = False):
+    """Gradients (dq, dk, dv) of the forward for the upstream gradient dout."""
+    q, k, v, o, dout = (t.contiguous() for t in (q, k, v, o, dout))
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    backward_into(q, k, v, o, lse.contiguous(), dout, dq, dk, dv, scale=scale, causal=causal)
+    return dq, dk, dv
 
 
 def check_device_status(stream: torch.cuda.Stream | None = None) -> None:

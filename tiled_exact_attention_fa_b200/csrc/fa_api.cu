@@ -16,6 +16,7 @@
 
 #include "fa.h"
 #include "fa_testing.h"
+#include "fa_bwd_tc.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
@@ -55,6 +56,7 @@ struct DeviceState {
     int cc_major = 0;
     bool smem_raised[4] = {false, false, false, false};
     bool decode_smem_raised[8] = {false, false, false, false, false, false, false, false};
+    bool bwd_smem_raised[8] = {false, false, false, false, false, false, false, false};
 };
 
 constexpr int kMaxDevices = 64;
@@ -727,4 +729,106 @@ extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, f
     if (d == 128) return one ? launch_decode<float, 128, 1>(st, 4, p, pl, s)
                              : launch_decode<float, 128, fa::dec::kMaxQ>(st, 5, p, pl, s);
     return one ? launch_decode<float, 64, 1>(st, 6, p, pl, s) : launch_decode<float, 64, fa::dec::kMaxQ>(st, 7, p, pl, s);
+}
+
+// ---------------------------------------------------------------------------
+// fa_bwd: gradients (see fa_bwd_tc.cuh).  Workspace: D = rowsum(dO * O),
+// [B*H][N] fp32.
+namespace {
+
+template <int D, bool kCausal>
+int launch_bwd(DeviceState* st, int slot, const void* q, const void* k, const void* v, const void* o,
+               const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dsum, int64_t bh,
+               int64_t n, float scale, cudaStream_t s) {
+    using L = fa::bwd::Layout<D>;
+    auto kdq = fa::bwd::fa_bwd_dq_kernel<D, kCausal>;
+    auto kkv = fa::bwd::fa_bwd_dkdv_kernel<D, kCausal>;
+    cudaError_t e;
+    if (!st->bwd_smem_raised[slot]) {
+        if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes)) != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->bwd_smem_raised[slot] = true;
+    }
+    const int64_t rows = bh * n;
+    fa::bwd::fa_bwd_dot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), dsum, rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the backward row-dot kernel");
+    CUtensorMap tq, tk, tv, tdo;
+    int rc;
+    if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK || (rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK ||
+        (rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK || (rc = encode_tile_map(&tdo, dout, bh, n, D)) != FA_OK)
+        return rc;
+    fa::bwd::Params p;
+    p.lse = lse;
+    p.dsum = dsum;
+    p.status = st->status;
+    p.n = static_cast<int>(n);
+    p.nblocks = static_cast<int>((n + fa::bwd::kBlock - 1) / fa::bwd::kBlock);
+    p.scale = scale;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    dim3 grid(static_cast<unsigned>(p.nblocks), static_cast<unsigned>(bh));
+    p.out0 = static_cast<__nv_bfloat16*>(dq);
+    p.out1 = nullptr;
+    kdq<<<grid, fa::bwd::kThreads, L::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the dQ kernel");
+    p.out0 = static_cast<__nv_bfloat16*>(dv);
+    p.out1 = static_cast<__nv_bfloat16*>(dk);
+    kkv<<<grid, fa::bwd::kThreads, L::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the dK/dV kernel");
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t fa_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    if (B < 1 || H < 1 || N < 1 || d < 1 || B > (int64_t{1} << 24) / H || N > (int64_t{1} << 30)) return 0;
+    return round_up(static_cast<size_t>(B * H * N) * 4, 256);
+}
+
+extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+                      int causal, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    g_last_error.clear();
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
+        return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (dtype != FA_DTYPE_BF16) return fail(FA_ERR_UNSUPPORTED, "the backward pass takes bf16 tensors");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (N > (int64_t{1} << 30) || B > 65535 / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H or N too large");
+    const int64_t bh = B * H;
+    const size_t tb = static_cast<size_t>(bh * N * d * 2), lb = static_cast<size_t>(bh * N * 4);
+    const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+    if (!workspace || workspace_bytes < need) return fail(FA_ERR_INVALID_ARGUMENT, "workspace missing or too small");
+    auto mis = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16) || mis(dout, 16) || mis(dq, 16) || mis(dk, 16) ||
+        mis(dv, 16) || mis(workspace, 16))
+        return fail(FA_ERR_INVALID_ARGUMENT, "tensors and workspace must be 16-byte aligned");
+    if (mis(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    const void* ins[6] = {q, k, v, o, dout, lse};
+    const size_t insz[6] = {tb, tb, tb, tb, tb, lb};
+    void* outs[4] = {dq, dk, dv, workspace};
+    const size_t outsz[4] = {tb, tb, tb, need};
+    for (int a = 0; a < 4; ++a) {
+        for (int b = 0; b < 6; ++b)
+            if (overlaps(outs[a], outsz[a], ins[b], insz[b]))
+                return fail(FA_ERR_INVALID_ARGUMENT, "an output or the workspace overlaps an input");
+        for (int b = a + 1; b < 4; ++b)
+            if (overlaps(outs[a], outsz[a], outs[b], outsz[b]))
+                return fail(FA_ERR_INVALID_ARGUMENT, "outputs overlap each other");
+    }
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the backward kernels need an sm_100 (B200-class) GPU");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* dsum = static_cast<float*>(workspace);
+    const bool c = causal != 0;
+    if (d == 128) return c ? launch_bwd<128, true>(st, 0, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s)
+                           : launch_bwd<128, false>(st, 1, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
+    return c ? launch_bwd<64, true>(st, 2, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s)
+             : launch_bwd<64, false>(st, 3, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
 }
