@@ -15,16 +15,17 @@
 //   * fa_bwd_dot_kernel: D = rowsum(dO * O), one warp per row;
 //   * fa_bwd_dq_kernel: one CTA per (head, 128-row query block) walks the KV
 //     blocks: S = Q K_j^T and dP = dO V_j^T into TMEM, the compute warps turn
-//     them into dS (bf16, written back over S), then dQ += dS K_j in TMEM;
+//     them into dS (bf16, into free TMEM columns), then dQ += dS K_j in TMEM;
 //   * fa_bwd_dkdv_kernel: one CTA per (head, 128-key block) walks the query
 //     blocks: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, the compute warps
 //     write P^T and dS^T (bf16) over them, then dV += P^T dO_i and
 //     dK += dS^T Q_i in TMEM.
 // S and dP are computed in both kernels (so dQ needs no atomics across
 // CTAs); that is 14 instead of 10 units of N^2 d work.  Roles per CTA: warps
-// 0-3 compute (one TMEM lane = one row per thread), warp 4 issues tcgen05.mma
-// from one elected lane, warp 5 streams tiles with TMA through a 4-slot
-// shared-memory ring.  All operand forms are the forward's: K-major
+// 0-7 compute (one TMEM lane = one row per thread; the two warps of a lane
+// quarter take one half of the 128 columns each), warp 8 issues
+// tcgen05.mma from one elected lane, warp 9 streams tiles with TMA through a
+// 4-slot shared-memory ring.  All operand forms are the forward's: K-major
 // shared-memory operands (Q, K, V, dO with d contiguous), MN-major B operands
 // for the products over rows (K, Q, dO as [rows][d]), and A from TMEM.
 // Every mbarrier wait is bounded (status word, abort flag, drain), as in the
@@ -42,10 +43,10 @@ namespace fa {
 namespace bwd {
 
 constexpr int kBlock = 128;       // rows (queries or keys) per tile
-constexpr int kComputeWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kComputeWarps = 8;  // two per TMEM lane quarter, one half of the columns each
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kSlots = 4;         // streamed tiles in flight
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -70,6 +71,7 @@ struct Layout {
     static constexpr uint32_t kTmemDP = 128;     // dP or dP^T; dS^T over its first 64 columns
     static constexpr uint32_t kTmemAcc0 = 256;   // dQ, or dV
     static constexpr uint32_t kTmemAcc1 = 256 + D;  // dK
+    static constexpr uint32_t kTmemDS = 384;         // dS of the dQ kernel (64 columns of bf16 pairs)
 };
 
 struct Params {
@@ -235,7 +237,7 @@ __device__ void mma_loop(const Common<D>& c, const fa::tc::Sync& sync, uint32_t 
             mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemS, c.slot_addr(ys), b > 0);   // dV += P^T dO
             mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc1, tmem + L::kTmemDP, c.slot_addr(xs), b > 0);  // dK += dS^T Q
         } else {
-            mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemS, c.slot_addr(xs), b > 0);   // dQ += dS K
+            mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemDS, c.slot_addr(xs), b > 0);  // dQ += dS K
         }
         commit(c.empty(xs));
         commit(c.empty(ys));
@@ -246,12 +248,13 @@ __device__ void mma_loop(const Common<D>& c, const fa::tc::Sync& sync, uint32_t 
     __syncwarp();
 }
 
-// Epilogue: 32 columns at a time of a TMEM accumulator (times `mul`) to bf16
-// global rows, one row per thread.
+// Epilogue: columns [col_begin, col_begin + D/2) of a TMEM accumulator (times
+// `mul`), 32 at a time, to bf16 global rows, one row per thread.
 template <int D>
-__device__ __forceinline__ void store_rows(uint32_t tmem_rows, __nv_bfloat16* row_ptr, bool valid, float mul) {
+__device__ __forceinline__ void store_rows(uint32_t tmem_rows, __nv_bfloat16* row_ptr, bool valid, float mul,
+                                           int col_begin) {
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = col_begin; c0 < col_begin + D / 2; c0 += 32) {
         uint32_t acc[32];
         ptx::tmem_ld32_wait(tmem_rows + c0, acc);
         uint32_t packed[16];
@@ -315,20 +318,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         mma_loop<D, false>(c, sync, tmem, nb);
     } else {
-        // one query row per thread: TMEM lane = row within the block
-        const int r = warp * 32 + lane;
+        // one query row per thread (TMEM lane = row within the block); the
+        // warp's half h of the key columns
+        const int q4 = warp & 3, h = warp >> 2;
+        const int r = q4 * 32 + lane;
         const int row = qb * kBlock + r;
         const bool valid = row < p.n;
         const float lse2 = valid ? p.lse[static_cast<int64_t>(bh) * p.n + row] * kLog2e : 0.f;
         const float drow = valid ? p.dsum[static_cast<int64_t>(bh) * p.n + row] : 0.f;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * warp) << 16;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
         bool ok = true;
         for (int j = 0; j < nb && ok; ++j) {
             ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.s_full(), j & 1));
             if (!ok) break;
             ptx::tc_fence_after_sync();
 #pragma unroll
-            for (int c0 = 0; c0 < kBlock; c0 += 32) {
+            for (int cl = 0; cl < kBlock / 2; cl += 32) {
+                const int c0 = h * (kBlock / 2) + cl;
                 uint32_t sv[32], gv[32];
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemS + c0, sv);
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemDP + c0, gv);
@@ -345,8 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ds[e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
                 }
-                // dS over the S columns already read (in-order: c0/2 + 16 <= c0 + 32)
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemS + c0 / 2, ds);
+                ptx::tmem_st16(tmem + lane_addr + L::kTmemDS + c0 / 2, ds);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before_sync();
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             ptx::tc_fence_after_sync();
             store_rows<D>(tmem + lane_addr + L::kTmemAcc0, p.out0 + (static_cast<int64_t>(bh) * p.n + row) * D, valid,
-                          p.scale);
+                          p.scale, h * (D / 2));
         }
     }
     ptx::tc_fence_before_sync();
@@ -419,17 +424,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         mma_loop<D, true>(c, sync, tmem, nb);
     } else {
-        // one key row per thread: TMEM lane = key within the block
-        const int r = warp * 32 + lane;
+        // one key row per thread (TMEM lane = key within the block); the
+        // warp's half h of the query columns
+        const int q4 = warp & 3, h = warp >> 2;
+        const int r = q4 * 32 + lane;
         const int key = kb * kBlock + r;
         const bool kvalid = key < p.n;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * warp) << 16;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
         bool ok = true;
         for (int b = 0; b < nb && ok; ++b) {
             const int i = i_begin + b;
-            // this query block's statistics, shared by the 128 compute threads
+            // this query block's statistics, shared by the compute threads
             asm volatile("bar.sync 1, %0;" ::"r"(32 * kComputeWarps) : "memory");
-            {
+            if (h == 0) {
                 const int qrow = i * kBlock + r;
                 const bool qv = qrow < p.n;
                 lse2_sm[r] = qv ? p.lse[static_cast<int64_t>(bh) * p.n + qrow] * kLog2e : 0.f;
@@ -439,12 +446,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.s_full(), b & 1));
             if (!ok) break;
             ptx::tc_fence_after_sync();
+            uint32_t pp[2][16], ds[2][16];
 #pragma unroll
-            for (int c0 = 0; c0 < kBlock; c0 += 32) {
+            for (int ci = 0; ci < 2; ++ci) {
+                const int c0 = h * (kBlock / 2) + ci * 32;
                 uint32_t sv[32], gv[32];
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemS + c0, sv);
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemDP + c0, gv);
-                uint32_t pp[16], ds[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     float p2[2], d2[2];
@@ -456,12 +464,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p2[u] = use ? ptx::ex2(__uint_as_float(sv[e + u]) * p.scale_log2 - lse2_sm[qc]) : 0.f;
                         d2[u] = p2[u] * (__uint_as_float(gv[e + u]) - dsum_sm[qc]);
                     }
-                    pp[e >> 1] = ptx::pack_bf16x2(p2[0], p2[1]);
-                    ds[e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
+                    pp[ci][e >> 1] = ptx::pack_bf16x2(p2[0], p2[1]);
+                    ds[ci][e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
                 }
-                // P^T over S^T and dS^T over dP^T, over columns already read
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemS + c0 / 2, pp);
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemDP + c0 / 2, ds);
+            }
+            // P^T goes over S^T and dS^T over dP^T: the second warp's results
+            // land on columns the first warp reads, so the pair meets first
+            asm volatile("bar.sync %0, 64;" ::"r"(2 + q4) : "memory");
+#pragma unroll
+            for (int ci = 0; ci < 2; ++ci) {
+                const int c0 = h * (kBlock / 2) + ci * 32;
+                ptx::tmem_st16(tmem + lane_addr + L::kTmemS + c0 / 2, pp[ci]);
+                ptx::tmem_st16(tmem + lane_addr + L::kTmemDP + c0 / 2, ds[ci]);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before_sync();
@@ -471,8 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             ptx::tc_fence_after_sync();
             const int64_t off = (static_cast<int64_t>(bh) * p.n + key) * D;
-            store_rows<D>(tmem + lane_addr + L::kTmemAcc0, p.out0 + off, kvalid, 1.f);      // dV
-            store_rows<D>(tmem + lane_addr + L::kTmemAcc1, p.out1 + off, kvalid, p.scale);  // dK
+            store_rows<D>(tmem + lane_addr + L::kTmemAcc0, p.out0 + off, kvalid, 1.f, h * (D / 2));      // dV
+            store_rows<D>(tmem + lane_addr + L::kTmemAcc1, p.out1 + off, kvalid, p.scale, h * (D / 2));  // dK
         }
     }
     ptx::tc_fence_before_sync();
