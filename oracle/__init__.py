@@ -73,6 +73,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     b.restype = ctypes.c_int
     b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    m = lib.oracle_lse_merge
+    m.restype = ctypes.c_int
+    m.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int64] * 3 + [ctypes.c_void_p] * 2
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_version.restype = ctypes.c_int
     return lib
@@ -165,3 +168,23 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool, lib=None):
     if rc != 0:
         raise RuntimeError(f"oracle_attention_bwd failed with code {rc}")
     return dq, dk, dv
+
+
+def lse_merge(o_parts, lse_parts, lib=None):
+    """Combine per-key-set results: o_parts [P, ..., d], lse_parts [P, ...]
+    (same leading shape) -> (o, lse) over the union of the key sets, fp64."""
+    lib = lib or load()
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float32)
+    lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float32)
+    P = o_parts.shape[0]
+    lead = o_parts.shape[1:-1]
+    d = o_parts.shape[-1]
+    if lse_parts.shape != (P,) + lead:
+        raise ValueError("lse_parts must match o_parts without its last axis")
+    rows = int(np.prod(lead)) if lead else 1
+    o = np.empty(lead + (d,), dtype=np.float64)
+    lse = np.empty(lead, dtype=np.float64)
+    rc = lib.oracle_lse_merge(o_parts.ctypes.data, lse_parts.ctypes.data, P, rows, d, o.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_lse_merge failed with code {rc}")
+    return o, lse

@@ -324,3 +324,43 @@ int oracle_attention_bwd(const float* q, const float* k, const float* v, const f
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * oracle_lse_merge -- combine attention results computed over disjoint key
+ * sets into the result over their union.  Each part i gives, per query row,
+ * o_i = sum_j exp(s_j - lse_i) v_j / 1 over its keys and lse_i = ln sum_j
+ * exp(s_j) over its keys; the union's softmax is then
+ *     lse = ln sum_i exp(lse_i),   o = sum_i exp(lse_i - lse) o_i
+ * -- the same identity the online softmax applies tile by tile
+ * ("FlashAttention, Playable", EP 04: rescale what was accumulated by the
+ * change of the running max), applied to whole partial results.  A part
+ * with lse_i = -inf (no key) contributes nothing.
+ *   o_parts: [parts][rows][d] fp32     lse_parts: [parts][rows] fp32
+ *   o: [rows][d] fp64                  lse: [rows] fp64
+ */
+int oracle_lse_merge(const float* o_parts, const float* lse_parts, int64_t parts, int64_t rows, int64_t d,
+                     double* o, double* lse) {
+    if (!o_parts || !lse_parts || !o || !lse || parts <= 0 || rows <= 0 || d <= 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double big = -INFINITY;
+        for (int64_t i = 0; i < parts; ++i) {
+            const double x = (double)lse_parts[i * rows + r];
+            if (x > big) big = x;
+        }
+        double tot = 0.0;
+        for (int64_t t = 0; t < d; ++t) o[r * d + t] = 0.0;
+        if (big == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        for (int64_t i = 0; i < parts; ++i) {
+            const double w = exp((double)lse_parts[i * rows + r] - big);
+            tot += w;
+            for (int64_t t = 0; t < d; ++t) o[r * d + t] += w * (double)o_parts[(i * rows + r) * d + t];
+        }
+        for (int64_t t = 0; t < d; ++t) o[r * d + t] /= tot;
+        lse[r] = big + log(tot);
+    }
+    return 0;
+}

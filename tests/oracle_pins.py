@@ -437,6 +437,37 @@ def pin_bwd_invariants(lib):
             np.testing.assert_allclose(c, 2 * a - 3 * b, atol=1e-11)
 
 
+# ------------------------------------------------- merging partial results
+def pin_merge_is_attention_over_the_union(lib):
+    """Attention over a key set split into parts, merged by log-sum-exp,
+    equals attention over the whole set (the forward oracle on the keys of
+    each part, then the merge, against the forward oracle on all keys), for
+    uneven parts and a part whose keys are all masked for some rows."""
+    B, H, N, d = 1, 2, 50, 8
+    q, k, v = (_rand((B, H, N, d), 110 + i) for i in range(3))
+    o_ref, lse_ref = _run(lib, q, k, v, 0.4, False)
+    bounds = [0, 7, 30, 50]
+    parts_o, parts_l = [], []
+    for a, b in zip(bounds, bounds[1:]):
+        # queries against the keys [a, b): the decode oracle with nq = N and no mask
+        o_p, l_p = oracle.attention_decode(q, k[:, :, a:b], v[:, :, a:b], 0.4, False, lib=lib)
+        parts_o.append(o_p.astype(np.float32))
+        parts_l.append(l_p.astype(np.float32))
+    o, lse = oracle.lse_merge(np.stack(parts_o), np.stack(parts_l), lib=lib)
+    # the parts were rounded to fp32 before the merge: agreement to fp32 precision
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=2e-6)
+    # a part with no usable key (lse = -inf) changes nothing
+    o2, lse2 = oracle.lse_merge(np.stack(parts_o + [np.full_like(parts_o[0], 7.0)]),
+                                np.stack(parts_l + [np.full_like(parts_l[0], -np.inf)]), lib=lib)
+    np.testing.assert_array_equal(o2, o)
+    np.testing.assert_array_equal(lse2, lse)
+    # one part is the identity
+    o3, lse3 = oracle.lse_merge(np.stack(parts_o[:1]), np.stack(parts_l[:1]), lib=lib)
+    np.testing.assert_allclose(o3, parts_o[0], rtol=0, atol=1e-7)
+    np.testing.assert_allclose(lse3, parts_l[0], rtol=0, atol=1e-6)
+
+
 BWD_PINS = [pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants]
 
 DECODE_PINS = [pin_decode_hand_worked, pin_decode_closed_forms, pin_decode_is_the_last_rows_of_prefill,
@@ -446,4 +477,4 @@ ALL_PINS = [
     pin_hand_worked, pin_q_zero_mean_of_v, pin_single_key, pin_causal_row0, pin_affine_v,
     pin_key_permutation, pin_future_keys_ignored, pin_softmax_shift, pin_lse_bounds,
     pin_row_subset, pin_online_ledger, pin_torch_sdpa,
-] + DECODE_PINS + BWD_PINS
+] + DECODE_PINS + BWD_PINS + [pin_merge_is_attention_over_the_union]

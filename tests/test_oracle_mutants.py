@@ -49,6 +49,10 @@ MUTANTS = [
     ("bwd_dv_from_p_not_transposed", "av += pm[r * n + c] * (double)gh[r * d + t];",
      "av += pm[c * n + r] * (double)gh[r * d + t];"),
     ("bwd_mask_off", "if (causal && c > r) {", "if (0 && causal && c > r) {"),
+    ("merge_without_max", "const double w = exp((double)lse_parts[i * rows + r] - big);",
+     "const double w = exp((double)lse_parts[i * rows + r]);"),
+    ("merge_lse_without_max", "lse[r] = big + log(tot);", "lse[r] = log(tot);"),
+    ("merge_not_normalised", "for (int64_t t = 0; t < d; ++t) o[r * d + t] /= tot;", ""),
     ("bwd_dp_with_k", "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)vh[c * d + t];",
      "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)kh[c * d + t];"),
 ]
