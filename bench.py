@@ -15,6 +15,10 @@ slowest rank's.
 `--impl reference` times the fp64 CPU oracle (test infrastructure, the
 deliberately slow plain definition) on a bounded sample of the same workload.
 
+`--path ring` measures the sequence-parallel forward (ring of K/V chunks,
+partial results merged by log-sum-exp): under torchrun the real ring over
+NCCL, each rank holding one chunk of one sequence (strong scaling); on one
+GPU the same schedule emulated for --ring-chunks ranks, one after another.
 `--path backward` measures fa_bwd (dq, dk, dv from the saved lse) on the same
 workload, counting the customary 2.5x the forward's FLOPs.  `--path decode`
 measures the generation step instead (fa_decode: new queries
@@ -59,7 +63,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
-    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward"])
+    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward", "ring"])
+    ap.add_argument("--ring-chunks", type=int, default=4,
+                    help="--path ring on one GPU: sequence chunks emulated one rank after another")
     ap.add_argument("--decode-workload", default=W.DECODE_HEADLINE.name, choices=sorted(W.DECODE_BY_NAME))
     return ap.parse_args()
 
@@ -617,8 +623,78 @@ def run_backward(a, w: W.Workload):
     return 0
 
 
+RING_METRIC = "sequence-parallel attention fwd TFLOPS (bf16, d=128, N=8K causal; chunks merged by log-sum-exp)"
+
+
+def run_ring(a, w: W.Workload):
+    import tiled_exact_attention_fa_b200 as fa
+    from tiled_exact_attention_fa_b200 import ring
+
+    rank, local_rank, world = fdist.env_world()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        fdist.init("nccl", timeout_s=300)
+    q, k, v = (x.to(dev) for x in W.make_inputs(w))  # the whole sequence, same on every rank
+    chunks = world if world > 1 else a.ring_chunks
+    if w.N % chunks:
+        raise SystemExit("the sequence must split into equal chunks")
+    n = w.N // chunks
+    sl = slice(rank * n, (rank + 1) * n)
+    ql, kl, vl = (t[:, :, sl].contiguous() for t in (q, k, v))
+    stream = torch.cuda.current_stream(dev)
+    flops = accounting.attention_flops(w.B, w.H, w.N, w.d, w.causal)
+
+    def step():
+        if world > 1:
+            return ring.ring_attention(ql, kl, vl, causal=w.causal, scale=w.scale)
+        return ring.ring_attention_emulated(q, k, v, chunks, causal=w.causal, scale=w.scale)
+
+    for _ in range(a.warmup):
+        step()
+    fa.check_device_status()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
+        fdist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(a.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        fdist.barrier(dev)
+    fa.check_device_status()
+    ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.steps
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, peak_sus, _, peak_kind = measured_peaks()
+    line = {"metric": RING_METRIC, "unit": UNIT, "value": tf, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                       "seed": w.seed, "chunks": chunks,
+                       "mode": "ring over NCCL, one chunk per rank" if world > 1 else
+                       f"{chunks} ranks emulated one after another on one GPU",
+                       "flop_per_step": flops},
+            "roofline": {"bound": "tensor", "achieved": tf / world, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / world / peak, "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
+                         "traffic": None, "kernel": "fa_fwd_bf16_kernel per chunk pair + fa_merge_kernel"},
+            "clocks": clocks.summary(),
+            "gpu_launches": a.steps * (chunks * (chunks + 1) // 2 + chunks if w.causal else chunks * chunks + chunks)
+            // (world if world > 1 else 1)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        fdist.barrier(dev)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     a = parse()
+    if a.path == "ring":
+        return run_ring(a, W.BY_NAME[a.workload])
     if a.path == "backward":
         return run_backward(a, W.BY_NAME[a.workload])
     if a.path == "decode":

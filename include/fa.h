@@ -210,6 +210,24 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 size_t fa_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
 /*
+ * fa_merge -- combine attention results computed over disjoint key sets into
+ * the result over their union, per query row:
+ *     lse = ln sum_i exp(lse_i),   o = sum_i exp(lse_i - lse) o_i
+ * (the online softmax's rescale -- "FlashAttention, Playable", EP 04 --
+ * applied to whole partial results; the combining step of a
+ * sequence-parallel forward, where each rank attends to every key chunk).
+ *   o_parts    device, [parts][rows][d] of `dtype` (each part as fa_fwd or
+ *              fa_decode wrote it); lse_parts device, [parts][rows] fp32.  A
+ *              part with lse = -inf for a row (no usable key) adds nothing.
+ *   o, lse     device, [rows][d] of `dtype` and [rows] fp32; rows with no
+ *              usable key in any part get o = 0 and lse = -inf.
+ *   d 64 or 128; dtype FA_DTYPE_BF16 or FA_DTYPE_F32.  Alignment 16 bytes
+ *   (lse arrays 4); outputs must not overlap inputs.  Asynchronous on stream.
+ */
+int fa_merge(const void* o_parts, const float* lse_parts, int64_t parts, int64_t rows, int64_t d,
+             void* o, float* lse, int dtype, void* stream);
+
+/*
  * fa_check_device_status -- synchronise `stream`, then read and clear the
  * library's device status word for the current device.  Returns FA_OK,
  * FA_ERR_DEVICE_TIMEOUT when a kernel launched by this library gave up on a

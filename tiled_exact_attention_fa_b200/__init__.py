@@ -42,6 +42,8 @@ _SIGNATURES = {
     "fa_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int64] * 4 +
                [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 4),
+    "fa_merge": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
@@ -267,6 +269,25 @@ def backward(q, k, v, o, lse, dout, *, scale: float | None = None, causal: bool 
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     backward_into(q, k, v, o, lse.contiguous(), dout, dq, dk, dv, scale=scale, causal=causal)
     return dq, dk, dv
+
+
+def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, *, stream: torch.cuda.Stream | None = None):
+    """Combine results over disjoint key sets (fa_merge): o_parts [P, ..., d]
+    and lse_parts [P, ...] CUDA tensors -> (o [..., d], lse [...])."""
+    if o_parts.dtype not in _DTYPES or lse_parts.dtype != torch.float32:
+        raise TypeError("o_parts must be bf16 or fp32 and lse_parts fp32")
+    if lse_parts.shape != o_parts.shape[:-1] or not (o_parts.is_cuda and lse_parts.is_cuda):
+        raise ValueError("o_parts [P, ..., d] and lse_parts [P, ...] on the GPU")
+    o_parts, lse_parts = o_parts.contiguous(), lse_parts.contiguous()
+    P, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    o = torch.empty(o_parts.shape[1:], dtype=o_parts.dtype, device=o_parts.device)
+    lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    with torch.cuda.device(o_parts.device):
+        s = (stream or torch.cuda.current_stream(o_parts.device)).cuda_stream
+        _check(int(library().fa_merge(o_parts.data_ptr(), lse_parts.data_ptr(), P, rows, d, o.data_ptr(),
+                                      lse.data_ptr(), _DTYPES[o_parts.dtype], s)))
+    return o, lse
 
 
 def check_device_status(stream: torch.cuda.Stream | None = None) -> None:

@@ -18,6 +18,7 @@
 #include "fa_testing.h"
 #include "fa_bwd_tc.cuh"
 #include "fa_decode.cuh"
+#include "fa_merge.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 
@@ -831,4 +832,46 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
                            : launch_bwd<128, false>(st, 1, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
     return c ? launch_bwd<64, true>(st, 2, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s)
              : launch_bwd<64, false>(st, 3, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
+}
+
+// ---------------------------------------------------------------------------
+// fa_merge: attention results over disjoint key sets -> the result over their
+// union (see fa_merge.cuh).
+extern "C" int fa_merge(const void* o_parts, const float* lse_parts, int64_t parts, int64_t rows, int64_t d,
+                        void* o, float* lse, int dtype, void* stream) {
+    g_last_error.clear();
+    if (!o_parts || !lse_parts || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (parts < 1 || rows < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "parts, rows and d must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (parts > 65536 || rows > (int64_t{1} << 40) / parts) return fail(FA_ERR_INVALID_ARGUMENT, "sizes too large");
+    const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
+    auto mis = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(o_parts, 16) || mis(o, 16)) return fail(FA_ERR_INVALID_ARGUMENT, "o_parts and o must be 16-byte aligned");
+    if (mis(lse_parts, 4) || mis(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse arrays must be 4-byte aligned");
+    const size_t ob = static_cast<size_t>(rows * d * elem), lb = static_cast<size_t>(rows * 4);
+    if (overlaps(o, ob, o_parts, ob * parts) || overlaps(o, ob, lse_parts, lb * parts) || overlaps(o, ob, lse, lb) ||
+        overlaps(lse, lb, o_parts, ob * parts) || overlaps(lse, lb, lse_parts, lb * parts))
+        return fail(FA_ERR_INVALID_ARGUMENT, "outputs overlap the inputs");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+    const int np = static_cast<int>(parts);
+    if (dtype == FA_DTYPE_BF16) {
+        if (d == 128)
+            fa::merge::fa_merge_kernel<__nv_bfloat16, 128><<<blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(o_parts), lse_parts, np, rows, static_cast<__nv_bfloat16*>(o), lse);
+        else
+            fa::merge::fa_merge_kernel<__nv_bfloat16, 64><<<blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(o_parts), lse_parts, np, rows, static_cast<__nv_bfloat16*>(o), lse);
+    } else {
+        if (d == 128)
+            fa::merge::fa_merge_kernel<float, 128><<<blocks, 256, 0, s>>>(
+                static_cast<const float*>(o_parts), lse_parts, np, rows, static_cast<float*>(o), lse);
+        else
+            fa::merge::fa_merge_kernel<float, 64><<<blocks, 256, 0, s>>>(
+                static_cast<const float*>(o_parts), lse_parts, np, rows, static_cast<float*>(o), lse);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the merge kernel");
+    return FA_OK;
 }
