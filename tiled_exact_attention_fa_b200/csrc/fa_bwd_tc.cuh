@@ -61,8 +61,8 @@ struct Layout {
     static constexpr int kBOff = kTileBytes;                        // resident tile B (dO or V)
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    // a_full, b_full, full[S], empty[S], s_full, p_full, done, drain
-    static constexpr int kNumBars = 2 + 2 * kSlots + 4;
+    // a_full, b_full, full[S], empty[S], s_full, p_full, done, drain, sdp_free, p_full_odd
+    static constexpr int kNumBars = 2 + 2 * kSlots + 6;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kVecOff = (kMiscOff + 16 + 15) & ~15;      // float[2][kBlock] (dK/dV kernel)
     static constexpr int kBytes = kVecOff + 2 * kBlock * 4;
@@ -71,7 +71,7 @@ struct Layout {
     static constexpr uint32_t kTmemDP = 128;     // dP or dP^T; dS^T over its first 64 columns
     static constexpr uint32_t kTmemAcc0 = 256;   // dQ, or dV
     static constexpr uint32_t kTmemAcc1 = 256 + D;  // dK
-    static constexpr uint32_t kTmemDS = 384;         // dS of the dQ kernel (64 columns of bf16 pairs)
+    static constexpr uint32_t kTmemDS = 384;         // dS of the dQ kernel: two buffers of 64 columns
 };
 
 struct Params {
@@ -118,6 +118,12 @@ struct Common {
     __device__ uint32_t p_full() const { return bar0 + 8u * (3 + 2 * kSlots); }
     __device__ uint32_t done() const { return bar0 + 8u * (4 + 2 * kSlots); }
     __device__ uint32_t drain() const { return bar0 + 8u * (5 + 2 * kSlots); }
+    __device__ uint32_t sdp_free() const { return bar0 + 8u * (6 + 2 * kSlots); }
+    // the dQ kernel's dS(j) is signalled on p_full for even j and on this one
+    // for odd j: the compute warps may finish dS(j+1) before the MMA warp has
+    // observed dS(j), and one barrier would then complete two phases unseen
+    __device__ uint32_t p_full_odd() const { return bar0 + 8u * (7 + 2 * kSlots); }
+    __device__ uint32_t p_full_of(int j) const { return (j & 1) ? p_full_odd() : p_full(); }
     __device__ uint32_t slot_addr(int s) const { return base + L::kRingOff + s * L::kTileBytes; }
 };
 
@@ -197,6 +203,73 @@ __device__ __forceinline__ void mma_tmem_by_tile(bool leader, uint32_t d_tmem, u
     for (int ks = 0; ks < kBlock / 16; ++ks)
         if (leader)
             ptx::mma_ts(d_tmem, a_tmem + ks * 8, bd + ((ks * 16 * 128) >> 4), idesc, (accumulate || ks > 0) ? 1u : 0u);
+}
+
+// The dQ kernel's MMA loop, pipelined: as soon as the compute warps have
+// read S(j) and dP(j) (sdp_free), S(j+1) and dP(j+1) are issued over them,
+// so these products run while dS(j) is computed; dS alternates between two
+// TMEM buffers, and dQ += dS(j) K_j follows once dS(j) is in place.  In-order
+// execution makes the reuse safe: dQ(j) is issued before S(j+2), so when the
+// compute warps see S(j+2) complete, dQ(j) has read dS buffer j & 1.
+template <int D>
+__device__ void mma_loop_dq(const Common<D>& c, const fa::tc::Sync& sync, uint32_t tmem, int nb) {
+    using L = Layout<D>;
+    const bool leader = ptx::elect_one();
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, fa::tc::wait_bar(sync, bar, parity));
+    };
+    auto commit = [&](uint32_t bar) {
+        if (leader) ptx::mma_commit(bar);
+    };
+    int slot = 0;
+    uint32_t phase = 0;
+    // the next (K_j, V_j) pair of ring slots
+    auto take = [&](int& xs, uint32_t& xp, int& ys, uint32_t& yp) {
+        xs = slot;
+        ys = slot + 1;
+        xp = yp = phase;
+        slot = (slot + 2) % kSlots;
+        if (slot < 2) phase ^= 1;
+    };
+    auto issue_sdp = [&](int xs, int ys) {
+        mma_rows_by_rows<D>(leader, tmem + L::kTmemS, c.base + L::kAOff, c.slot_addr(xs));   // S = Q K^T
+        mma_rows_by_rows<D>(leader, tmem + L::kTmemDP, c.base + L::kBOff, c.slot_addr(ys));  // dP = dO V^T
+        commit(c.s_full());
+        commit(c.empty(ys));  // V_j is done once dP is
+    };
+    bool ok = wait_all(c.a_full(), 0) && wait_all(c.b_full(), 0);
+    int xs, ys;
+    uint32_t xp, yp;
+    take(xs, xp, ys, yp);
+    ok = ok && wait_all(c.full(xs), xp) && wait_all(c.full(ys), yp);
+    if (ok) {
+        ptx::tc_fence_after_sync();
+        issue_sdp(xs, ys);
+    }
+    int kslot = xs;
+    for (int j = 0; j < nb && ok; ++j) {
+        ok = wait_all(c.sdp_free(), j & 1);
+        if (!ok) break;
+        int next_k = -1;
+        if (j + 1 < nb) {
+            take(xs, xp, ys, yp);
+            ok = wait_all(c.full(xs), xp) && wait_all(c.full(ys), yp);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            issue_sdp(xs, ys);
+            next_k = xs;
+        }
+        ok = wait_all(c.p_full_of(j), (j >> 1) & 1);
+        if (!ok) break;
+        ptx::tc_fence_after_sync();
+        mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemDS + 64 * (j & 1), c.slot_addr(kslot), j > 0);
+        commit(c.empty(kslot));  // K_j is done once dQ(j) is
+        kslot = next_k;
+    }
+    commit(c.done());
+    commit(c.drain());
+    fa::tc::drain_bar(sync, c.drain(), 0);
+    __syncwarp();
 }
 
 // The MMA warp's loop, shared by both kernels (A, B resident; streamed pairs
@@ -301,6 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(c.p_full(), 32 * kComputeWarps);
         ptx::mbar_init(c.done(), 1);
         ptx::mbar_init(c.drain(), 1);
+        ptx::mbar_init(c.sdp_free(), 32 * kComputeWarps);
+        ptx::mbar_init(c.p_full_odd(), 32 * kComputeWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -316,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
         produce<D>(c, sync, &tm_q, &tm_do, qb * kBlock, &tm_k, &tm_v, 0, nb, bh);
     } else if (warp == kMmaWarp) {
-        mma_loop<D, false>(c, sync, tmem, nb);
+        mma_loop_dq<D>(c, sync, tmem, nb);
     } else {
         // one query row per thread (TMEM lane = row within the block); the
         // warp's half h of the key columns
@@ -332,12 +407,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.s_full(), j & 1));
             if (!ok) break;
             ptx::tc_fence_after_sync();
+            const uint32_t ds_buf = L::kTmemDS + 64 * (j & 1);
 #pragma unroll
             for (int cl = 0; cl < kBlock / 2; cl += 32) {
                 const int c0 = h * (kBlock / 2) + cl;
                 uint32_t sv[32], gv[32];
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemS + c0, sv);
                 ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemDP + c0, gv);
+                if (cl + 32 == kBlock / 2) {
+                    // S(j) and dP(j) are in registers: the next pair may overwrite them
+                    ptx::tc_fence_before_sync();
+                    ptx::mbar_arrive(c.sdp_free());
+                }
                 uint32_t ds[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -351,11 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ds[e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
                 }
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemDS + c0 / 2, ds);
+                ptx::tmem_st16(tmem + lane_addr + ds_buf + c0 / 2, ds);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(c.p_full());
+            ptx::mbar_arrive(c.p_full_of(j));
         }
         if (ok) ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.done(), 0));
         if (ok) {
