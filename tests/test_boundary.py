@@ -187,3 +187,29 @@ def test_backward_rejected_before_cuda(lib):
     assert bwd(args[:6] + [A + 6 * NB + 8] + args[7:]) == fa.FA_ERR_INVALID_ARGUMENT  # misaligned
     assert lib.fa_bwd_workspace_bytes(2, 3, 1000, 128) >= 2 * 3 * 1000 * 4
     assert lib.fa_bwd_workspace_bytes(0, 3, 1000, 128) == 0
+
+
+def test_merge_rejected_before_cuda(lib):
+    def merge(op=A, lp=A + NB, parts=2, rows=10, d=128, o=A + 2 * NB, lse=A + 3 * NB, dtype=fa.FA_DTYPE_BF16):
+        return lib.fa_merge(op, lp, parts, rows, d, o, lse, dtype, None)
+
+    assert merge(op=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert merge(parts=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert merge(rows=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert merge(dtype=5) == fa.FA_ERR_INVALID_ARGUMENT
+    assert merge(d=32) == fa.FA_ERR_UNSUPPORTED
+    assert merge(o=A + 2 * NB + 4) == fa.FA_ERR_INVALID_ARGUMENT   # misaligned
+    assert merge(o=A + 64) == fa.FA_ERR_INVALID_ARGUMENT           # output inside the parts
+    assert lib.fa_last_error().decode() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_other_entries_need_a_gpu(lib):
+    # well-formed calls of the other entry points fail with a CUDA error on a
+    # machine without a GPU: never a CPU result
+    assert lib.fa_decode(A, A + NB, A + 2 * NB, A + 3 * NB, A + 4 * NB, 1, 1, 1, 128, 128, 0.1, 0,
+                         fa.FA_DTYPE_BF16, None, 0, None) == fa.FA_ERR_CUDA
+    assert lib.fa_merge(A, A + NB, 2, 10, 128, A + 2 * NB, A + 3 * NB, fa.FA_DTYPE_BF16, None) == fa.FA_ERR_CUDA
+    ws = lib.fa_bwd_workspace_bytes(1, 1, 128, 128)
+    assert lib.fa_bwd(A, A + NB, A + 2 * NB, A + 3 * NB, A + 4 * NB, A + 5 * NB, A + 6 * NB, A + 7 * NB,
+                      A + 8 * NB, 1, 1, 128, 128, 0.1, 0, fa.FA_DTYPE_BF16, A + 9 * NB, ws, None) == fa.FA_ERR_CUDA
