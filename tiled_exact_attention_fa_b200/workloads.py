@@ -145,6 +145,8 @@ DECODE_WORKLOADS = [
     DecodeWorkload("bf16_decode_b1h8_q1_nk262144_d128", torch.bfloat16, 1, 8, 1, 262144, 128, True, 6),
     # four new tokens at once (speculative / chunked step), causal among them
     DecodeWorkload("bf16_decode_b8h32_q4_nk32768_d128", torch.bfloat16, 8, 32, 4, 32768, 128, True, 7),
+    # the same with a batch of 2 (1.07 GB of cache)
+    DecodeWorkload("bf16_decode_b2h32_q4_nk32768_d128", torch.bfloat16, 2, 32, 4, 32768, 128, True, 8),
 ]
 DECODE_BY_NAME = {w.name: w for w in DECODE_WORKLOADS}
 DECODE_HEADLINE = DECODE_BY_NAME["bf16_decode_b16h32_q1_nk16384_d128"]
