@@ -239,20 +239,20 @@ __global__ void __launch_bounds__(kThreads) fa_decode_kernel(const Params p) {
             const T* vt = kt + kTileKeys * D;
             const int key0 = key_begin + t * kTileKeys + warp * kKeysPerWarp;
             // This warp's 8 keys: the lane's slice of every K and V row (V
-            // rows past the cache end are zeroed so that p = 0 stays 0).
+            // rows past the cache end are zeroed so that p = 0 stays 0).  K
+            // rows are taken in a lane-dependent order, slot j holding key
+            // j ^ myk, so that the transposed butterfly below sends and keeps
+            // the same slots on every lane and needs no selects.
+            const int myk = (lane >> 2) & 7;
             float kx[kKeysPerWarp][kPer], vx[kKeysPerWarp][kPer];
 #pragma unroll
             for (int j = 0; j < kKeysPerWarp; ++j) {
-                load_slice<T, kPer>(kt + j * D, lane, kx[j]);
+                load_slice<T, kPer>(kt + (j ^ myk) * D, lane, kx[j]);
                 load_slice<T, kPer>(vt + j * D, lane, vx[j]);
                 if (key0 + j >= key_end)
 #pragma unroll
                     for (int e = 0; e < kPer; ++e) vx[j][e] = 0.f;
             }
-            // After the transposed butterfly below, lanes 4k .. 4k+3 hold the
-            // complete score of key k of the group.
-            const int myk = (lane >> 2) & 7;
-            const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
                 if (i >= nqc) break;
@@ -264,16 +264,17 @@ __global__ void __launch_bounds__(kThreads) fa_decode_kernel(const Params p) {
                     for (int e = 0; e < kPer; ++e) d0 = fmaf(qr[i][e], kx[j][e], d0);
                     part[j] = d0;
                 }
-                // reduce 8 partial sums over 32 lanes with 9 shuffles: each
-                // round keeps half of the keys and adds the partner's half
+                // Reduce 8 partial sums over 32 lanes with 9 shuffles.  The
+                // partner across lane bit 4 has myk ^ 4, so its slot j + 4 is
+                // this lane's key j ^ myk; likewise across bits 3 and 2.  After
+                // three rounds lanes 4k .. 4k+3 hold the quarter sums of key
+                // k, and two more complete it.
                 float w4[4], w2[2], sc;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    w4[j] = (b4 ? part[j + 4] : part[j]) + __shfl_xor_sync(0xffffffffu, b4 ? part[j] : part[j + 4], 16);
+                for (int j = 0; j < 4; ++j) w4[j] = part[j] + __shfl_xor_sync(0xffffffffu, part[j + 4], 16);
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    w2[j] = (b3 ? w4[j + 2] : w4[j]) + __shfl_xor_sync(0xffffffffu, b3 ? w4[j] : w4[j + 2], 8);
-                sc = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+                for (int j = 0; j < 2; ++j) w2[j] = w4[j] + __shfl_xor_sync(0xffffffffu, w4[j + 2], 8);
+                sc = w2[0] + __shfl_xor_sync(0xffffffffu, w2[1], 4);
                 sc += __shfl_xor_sync(0xffffffffu, sc, 2);
                 sc += __shfl_xor_sync(0xffffffffu, sc, 1);
                 // mask: past the cache, or (causal) past query i's position
