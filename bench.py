@@ -20,7 +20,10 @@ partial results merged by log-sum-exp): under torchrun the real ring over
 NCCL, each rank holding one chunk of one sequence (strong scaling); on one
 GPU the same schedule emulated for --ring-chunks ranks, one after another.
 `--path backward` measures fa_bwd (dq, dk, dv from the saved lse) on the same
-workload, counting the customary 2.5x the forward's FLOPs.  `--path decode`
+workload, counting the customary 2.5x the forward's FLOPs.  `--path fp8`
+measures fa_fwd_fp8 (E4M3 Q, K, V, bf16 O) on an E4M3 workload of the same
+shape (default e4m3_b2h32_n8192_d128_causal) against the measured bf16 peak
+times the nominal FP8/BF16 ratio of 2.  `--path decode`
 measures the generation step instead (fa_decode: new queries
 over a resident key/value cache, HBM-bound): the metric is the cache bytes
 read per second, against the measured HBM copy bandwidth.
@@ -63,7 +66,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
-    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward", "ring"])
+    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward", "ring", "fp8"])
     ap.add_argument("--ring-chunks", type=int, default=4,
                     help="--path ring on one GPU: sequence chunks emulated one rank after another")
     ap.add_argument("--decode-workload", default=W.DECODE_HEADLINE.name, choices=sorted(W.DECODE_BY_NAME))
@@ -92,7 +95,8 @@ def traffic_from_profile(w):
         return None
     with open(path) as f:
         d = json.load(f)
-    kind = "decode" if isinstance(w, W.DecodeWorkload) else "forward"
+    kind = ("decode" if isinstance(w, W.DecodeWorkload) else
+            "forward_fp8" if w.dtype == torch.float8_e4m3fn else "forward")
     if d.get("kernel_digest") != kernel_digest(kind):
         return None
     return d.get("dram_bytes_per_launch")
@@ -217,7 +221,7 @@ def run_reference(a, w: W.Workload):
         works.append(work)
     value = sum(works) / sum(times) / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "impl": "reference", "metric": FP8_METRIC if w.dtype == torch.float8_e4m3fn else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
@@ -325,6 +329,114 @@ def run_ours(a, w: W.Workload):
     if "cpu" in legs and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_leg(w, a.cpu_seconds)
 
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        fdist.barrier(dev)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+FP8_METRIC = "attention fwd TFLOPS (E4M3 Q/K/V, bf16 O, d=128) and % of B200 dense FP8 peak"
+FP8_DEFAULT = "e4m3_b2h32_n8192_d128_causal"
+
+
+def run_fp8(a, w: W.Workload):
+    """fa_fwd_fp8 on an E4M3 workload (inputs resident in HBM; e2e adds the
+    host-to-device copies of Q, K, V and the copy back of O and lse)."""
+    import tiled_exact_attention_fa_b200 as fa
+
+    rank, local_rank, world = fdist.env_world()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        fdist.init("nccl", timeout_s=300)
+    legs = set(a.legs.split(","))
+    wr = W.Workload(w.name, w.dtype, w.B, w.H, w.N, w.d, w.causal, w.seed + 1000 * rank, w.q_mult)
+    q_h, k_h, v_h = W.make_inputs(wr, pin=True)
+    q, k, v = (x.to(dev, non_blocking=True) for x in (q_h, k_h, v_h))
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = accounting.attention_flops(w.B, w.H, w.N, w.d, w.causal)
+    rows = w.B * w.H * w.N
+    in_bytes = 3 * rows * w.d
+    out_bytes = 2 * rows * w.d + 4 * rows
+    alg_bytes = in_bytes + out_bytes
+
+    def step():
+        fa.forward_fp8_into(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+
+    for _ in range(a.warmup):
+        step()
+    fa.check_device_status()
+    line = {"metric": FP8_METRIC, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic"}
+    line["config"] = {
+        "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "seed": w.seed,
+        "per_rank": "own seeded batch (seed + 1000*rank), no collective on the data path",
+        "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB, no flush between steps"
+        if in_bytes > L2_BYTES else "inputs smaller than L2: not flushed (not a valid headline)",
+        "flop_per_step": flops}
+    if "kernel" in legs:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
+            fdist.barrier(dev)
+            torch.cuda.synchronize(dev)
+            start.record(stream)
+            for _ in range(a.steps):
+                step()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+            fdist.barrier(dev)
+        fa.check_device_status()
+        ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.steps
+        tflops_rank = flops / (ms * 1e-3) / 1e12
+        peak, peak_sus, _, peak_kind = measured_peaks()
+        line["value"] = world * tflops_rank
+        line["ms_per_step"] = ms
+        line["roofline"] = {
+            "bound": "tensor", "achieved": tflops_rank, "peak": 2 * peak, "unit": "TFLOP/s",
+            "frac": tflops_rank / (2 * peak),
+            "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS) x 2, the nominal FP8/BF16 ratio",
+            "frac_of_sustained": tflops_rank / (2 * peak_sus),
+            "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
+            "kernel": f"fa_fwd_e4m3_kernel<{str(w.causal).lower()}>",
+            "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
+        line["clocks"] = clocks.summary()
+        line["gpu_launches"] = a.steps
+    if "e2e" in legs:
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q_h, k_h, v_h))
+            fa.forward_fp8_into(qd, kd, vd, o, lse, scale=w.scale, causal=w.causal)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fdist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(a.e2e_steps):
+            e2e_step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        fdist.barrier(dev)
+        e2e_ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.e2e_steps
+        line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
+                       "api": "pinned host Q, K, V copied in, tiled_exact_attention_fa_b200.forward_fp8_into "
+                              "(C ABI fa_fwd_fp8), O and lse copied back to pinned host memory"}
+        if "value" not in line:
+            line["value"] = line["e2e"]["value"]
+    if "cpu" in legs and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_leg(w, a.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -697,6 +809,13 @@ def main():
         return run_ring(a, W.BY_NAME[a.workload])
     if a.path == "backward":
         return run_backward(a, W.BY_NAME[a.workload])
+    if a.path == "fp8":
+        w = W.BY_NAME[a.workload]
+        if w.dtype != torch.float8_e4m3fn:
+            w = W.BY_NAME[FP8_DEFAULT]
+        if a.impl == "reference":
+            return run_reference(a, w)
+        return run_fp8(a, w)
     if a.path == "decode":
         wd = W.DECODE_BY_NAME[a.decode_workload]
         if a.impl == "reference":

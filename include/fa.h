@@ -115,6 +115,42 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
                    float scale, int causal, int dtype, void* stream);
 
 /*
+ * fa_fwd_fp8 -- the attention forward with 8-bit float inputs.
+ *
+ * The pages name low precision (FP8) as the step the third FlashAttention
+ * generation took on Hopper (Chapter 15 -- FlashAttention, "FlashAttention
+ * Evolution", FA-3) and fix nothing more.  Computed here, per head:
+ *
+ *     O = softmax(scale * (descale_q Q8)(descale_k K8)^T [causal]) (descale_v V8)
+ *
+ * with Q8, K8, V8 in OCP E4M3 (1 sign, 4 exponent, 3 mantissa bits, bias 7,
+ * largest finite 448; torch.float8_e4m3fn), Q K^T and P V on the tensor core
+ * with fp32 accumulation, P rounded to E4M3 (nearest) as the operand of P V,
+ * the running max and sum in fp32.  Q8 K8^T is exact in fp32 up to the
+ * accumulation order; the rounding of P is the one approximation, and each
+ * element of O lies within 2^-4 * sum_j p_j |v_j| + 2^-10 * sum_j |v_j| / l
+ * (+ the bf16 rounding of O) of the exact result, p_j the exact softmax
+ * weights and l = exp(lse - max_j s_j).
+ *
+ *   q, k, v  device, contiguous [B][H][N][d] one-byte E4M3.  16-byte aligned.
+ *   o        device, [B][H][N][d] bf16, written once per row.  16-byte aligned.
+ *   lse      device, [B][H][N] fp32 natural-log log-sum-exp of the scaled
+ *            scores (scale * descale_q * descale_k * q8 . k8).  4-byte aligned.
+ *   B, H, N  each >= 1; any N.
+ *   d        128 (others: FA_ERR_UNSUPPORTED).
+ *   scale, descale_q, descale_k, descale_v  finite floats; the product
+ *            scale * descale_q * descale_k must stay finite in fp32.
+ *   causal   as for fa_fwd.
+ *
+ * No output may overlap an input or the other output.  Asynchronous on
+ * `stream`; argument errors are reported before any CUDA call; device-side
+ * timeouts are reported by fa_check_device_status.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+               int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+               float descale_q, float descale_k, float descale_v, int causal, void* stream);
+
+/*
  * fa_fwd_host -- fa_fwd on buffers in host memory: the same operation,
  * arguments, layouts, results and errors, but q, k, v, o and lse may be host
  * pointers (page-locked memory, e.g. from cudaHostAlloc, for the copies to

@@ -213,3 +213,38 @@ def test_other_entries_need_a_gpu(lib):
     ws = lib.fa_bwd_workspace_bytes(1, 1, 128, 128)
     assert lib.fa_bwd(A, A + NB, A + 2 * NB, A + 3 * NB, A + 4 * NB, A + 5 * NB, A + 6 * NB, A + 7 * NB,
                       A + 8 * NB, 1, 1, 128, 128, 0.1, 0, fa.FA_DTYPE_BF16, A + 9 * NB, ws, None) == fa.FA_ERR_CUDA
+
+
+def call_fp8(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,
+             scale=0.1, dq=1.0, dk=1.0, dv=1.0, causal=0):
+    return lib.fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, dq, dk, dv, causal, None)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(lse=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(N=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(dq=float("inf")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(dv=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=1e30, dq=1e30, dk=1e30), fa.FA_ERR_INVALID_ARGUMENT),  # product overflows fp32
+    (dict(q=A + 8), fa.FA_ERR_INVALID_ARGUMENT),                       # misaligned
+    (dict(o=A + 2 * NB - 64), fa.FA_ERR_INVALID_ARGUMENT),             # bf16 o (2 bytes/elem) reaches v
+    (dict(lse=A + 3 * NB + 64), fa.FA_ERR_INVALID_ARGUMENT),           # lse inside o
+    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_rejected_before_cuda(lib, kwargs, code):
+    assert call_fp8(lib, **kwargs) == code
+    assert lib.fa_last_error().decode() != ""
+
+
+def test_fp8_output_is_twice_the_input_bytes(lib):
+    # o holds bf16: with q at A and o 16 KB below it, a 128 x 128 E4M3 head
+    # (16 KB) ends at q's start but its bf16 output (32 KB) runs into q
+    assert call_fp8(lib, o=A - 16384) == fa.FA_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_fp8_needs_a_gpu(lib):
+    assert call_fp8(lib) == fa.FA_ERR_CUDA

@@ -34,6 +34,8 @@ _SIGNATURES = {
                [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "fa_fwd_fp8": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
+                   [ctypes.c_float] * 4 + [ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                     [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "fa_decode": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 5 +
@@ -125,6 +127,45 @@ def _check_qkv(q, k, v, o, lse):
     for t in (q, k, v, o, lse):
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+
+
+def forward_fp8_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                     lse: torch.Tensor, *, descale_q: float = 1.0, descale_k: float = 1.0,
+                     descale_v: float = 1.0, scale: float | None = None, causal: bool = False,
+                     stream: torch.cuda.Stream | None = None) -> None:
+    """fa_fwd_fp8: q, k, v torch.float8_e4m3fn [B, H, N, 128] CUDA tensors,
+    each standing for its values times its descale factor; o bf16 [B, H, N,
+    128] and lse fp32 [B, H, N], caller-provided."""
+    if not (q.dtype == k.dtype == v.dtype == torch.float8_e4m3fn):
+        raise TypeError("q, k, v must be torch.float8_e4m3fn")
+    if o.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise TypeError("o must be bf16 and lse fp32")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or o.shape != q.shape:
+        raise ValueError("q, k, v, o must share one [B, H, N, d] shape")
+    if lse.shape != q.shape[:3]:
+        raise ValueError("lse must be [B, H, N]")
+    for t in (q, k, v, o, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("forward_fp8_into needs contiguous CUDA tensors")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    with torch.cuda.device(q.device):
+        _check(int(library().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                        B, H, N, d, float(scale), float(descale_q), float(descale_k),
+                                        float(descale_v), int(causal), s)))
+
+
+def forward_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, descale_q: float = 1.0,
+                descale_k: float = 1.0, descale_v: float = 1.0, scale: float | None = None,
+                causal: bool = False, stream: torch.cuda.Stream | None = None):
+    """(o bf16, lse fp32) of the attention over E4M3 inputs (see forward_fp8_into)."""
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    forward_fp8_into(q, k, v, o, lse, descale_q=descale_q, descale_k=descale_k, descale_v=descale_v,
+                     scale=scale, causal=causal, stream=stream)
+    return o, lse
 
 
 def forward_host_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,

@@ -1,7 +1,8 @@
 // fa_api.cu -- the C ABI (include/fa.h): argument checks, kernel choice,
 // TMA tensor-map encoding, persistent-grid sizing and launch on the caller's
 // stream.  All compute runs in the kernels of fa_fwd_tc.cuh (bf16, tensor
-// cores) and fa_fwd_simt.cuh (fp32, CUDA cores).
+// cores), fa_fwd_fp8_tc.cuh (E4M3, tensor cores), fa_fwd_simt.cuh (fp32,
+// CUDA cores) and the decode, backward and merge kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -19,6 +20,7 @@
 #include "fa_bwd_tc.cuh"
 #include "fa_decode.cuh"
 #include "fa_merge.cuh"
+#include "fa_fwd_fp8_tc.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 
@@ -58,6 +60,7 @@ struct DeviceState {
     bool smem_raised[4] = {false, false, false, false};
     bool decode_smem_raised[8] = {false, false, false, false, false, false, false, false};
     bool bwd_smem_raised[8] = {false, false, false, false, false, false, false, false};
+    bool fp8_smem_raised[2] = {false, false};
 };
 
 constexpr int kMaxDevices = 64;
@@ -874,4 +877,99 @@ extern "C" int fa_merge(const void* o_parts, const float* lse_parts, int64_t par
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the merge kernel");
     return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// fa_fwd_fp8: the forward with E4M3 inputs (see fa_fwd_fp8_tc.cuh).
+namespace {
+
+// 3-D view (d, N, B*H) of a [B*H][N][128] one-byte tensor, boxes of
+// 128 x 128 x 1 (one 128-byte swizzle panel); rows past N read as zeros.
+int encode_tile_map_u8(CUtensorMap* map, const void* ptr, int64_t bh, int64_t n) {
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(n * 128)};
+    cuuint32_t box[3] = {128, static_cast<cuuint32_t>(fa::tc::kBlockM), 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
+    return FA_OK;
+}
+
+template <bool kCausal>
+int launch_e4m3(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh,
+                int64_t n, double scale_qk, float o_scale, cudaStream_t stream) {
+    using L = fa::tc8::Layout;
+    auto kernel = fa::tc8::fa_fwd_e4m3_kernel<kCausal>;
+    if (!st->fp8_smem_raised[kCausal ? 0 : 1]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->fp8_smem_raised[kCausal ? 0 : 1] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = encode_tile_map_u8(&tq, q, bh, n)) != FA_OK) return rc;
+    if ((rc = encode_tile_map_u8(&tk, k, bh, n)) != FA_OK) return rc;
+    if ((rc = encode_tile_map_u8(&tv, v, bh, n)) != FA_OK) return rc;
+
+    fa::tc8::Params p;
+    p.base.o = static_cast<__nv_bfloat16*>(o);
+    p.base.lse = lse;
+    p.base.status = st->status;
+    p.base.sched = st->queues + 2 * (st->next_queue.fetch_add(1, std::memory_order_relaxed) % kQueues);
+    p.base.bh = static_cast<int>(bh);
+    p.base.n = static_cast<int>(n);
+    p.base.num_qblocks = static_cast<int>((n + fa::tc::kUnitRows - 1) / fa::tc::kUnitRows);
+    p.base.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
+    p.base.num_units = p.base.bh * p.base.num_qblocks;
+    p.base.scale_log2 = static_cast<float>(scale_qk * 1.4426950408889634);
+    p.base.skip_one_arrival = 0;
+    p.o_scale = o_scale;
+    const int grid = p.base.num_units < st->sm_count ? p.base.num_units : st->sm_count;
+    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the E4M3 attention kernel");
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                          int64_t N, int64_t d, float scale, float descale_q, float descale_k, float descale_v,
+                          int causal, void* stream) {
+    g_last_error.clear();
+    if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
+    if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
+    if (!std::isfinite(scale) || !std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v))
+        return fail(FA_ERR_INVALID_ARGUMENT, "scale and descale factors must be finite");
+    const double scale_qk = static_cast<double>(scale) * descale_q * descale_k;
+    if (!std::isfinite(static_cast<float>(scale_qk * 1.4426950408889634)))
+        return fail(FA_ERR_INVALID_ARGUMENT, "scale * descale_q * descale_k overflows fp32");
+    if (d != 128) return fail(FA_ERR_UNSUPPORTED, "the E4M3 forward takes head dim 128");
+    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    const int64_t bh = B * H;
+    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
+    if (bh * ((N + 255) / 256) > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
+    if (bh > (int64_t{1} << 62) / (N * d * 2)) return fail(FA_ERR_INVALID_ARGUMENT, "tensor size overflows");
+    const size_t in_bytes = static_cast<size_t>(bh * N * d), o_bytes = 2 * in_bytes;
+    const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
+    auto mis = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16))
+        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+    if (mis(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (overlaps(o, o_bytes, q, in_bytes) || overlaps(o, o_bytes, k, in_bytes) || overlaps(o, o_bytes, v, in_bytes) ||
+        overlaps(o, o_bytes, lse, lse_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
+    if (overlaps(lse, lse_bytes, q, in_bytes) || overlaps(lse, lse_bytes, k, in_bytes) ||
+        overlaps(lse, lse_bytes, v, in_bytes))
+        return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the E4M3 kernel needs an sm_100 (B200-class) GPU");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return causal ? launch_e4m3<true>(st, q, k, v, o, lse, bh, N, scale_qk, descale_v, s)
+                  : launch_e4m3<false>(st, q, k, v, o, lse, bh, N, scale_qk, descale_v, s);
 }

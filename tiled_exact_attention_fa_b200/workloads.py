@@ -38,7 +38,7 @@ class Workload:
 
     @property
     def dtype_name(self) -> str:
-        return {torch.float32: "f32", torch.bfloat16: "bf16"}[self.dtype]
+        return {torch.float32: "f32", torch.bfloat16: "bf16", torch.float8_e4m3fn: "e4m3"}[self.dtype]
 
     def describe(self) -> str:
         c = " causal" if self.causal else ""
@@ -55,7 +55,14 @@ WORKLOADS = [
     Workload("bf16_b1h16_n32768_d128_causal_q8", torch.bfloat16, 1, 16, 32768, 128, True, 4,
              q_mult=8.0, sample_rows=512),
 ]
-BY_NAME = {w.name: w for w in WORKLOADS}
+# The E4M3 forward (fa_fwd_fp8) on the shapes of the two large bf16 workloads:
+# the same fp32 draws, rounded to E4M3 (nearest; |x| < 448 for these draws, so
+# nothing saturates), with descale factors 1.
+FP8_WORKLOADS = [
+    Workload("e4m3_b4h16_n4096_d128", torch.float8_e4m3fn, 4, 16, 4096, 128, False, 2, sample_rows=512),
+    Workload("e4m3_b2h32_n8192_d128_causal", torch.float8_e4m3fn, 2, 32, 8192, 128, True, 3, sample_rows=512),
+]
+BY_NAME = {w.name: w for w in WORKLOADS + FP8_WORKLOADS}
 HEADLINE = BY_NAME["bf16_b2h32_n8192_d128_causal"]
 
 
