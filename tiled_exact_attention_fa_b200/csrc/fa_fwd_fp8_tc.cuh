@@ -13,28 +13,32 @@
 // written in bf16.  dq dk fold into the exponent's scale, dv into the final
 // normalisation, so the kernel never rescales an input.
 //
-// Same structure as the bf16 kernel (persistent CTAs, a producer warp, one
-// MMA-issuing warp, sixteen softmax warps over two 128-row query tiles, P
-// over S in TMEM), with what 8-bit operands change:
-//   * a 128 x 128 tile is one 128-byte swizzle panel (16 KB), so the K/V ring
-//     holds 8 slots in the shared memory that held 4 bf16 slots;
+// Same roles as the bf16 kernel (persistent CTAs, a producer warp, one
+// MMA-issuing warp, sixteen softmax warps over two 128-row query tiles), with
+// what 8-bit operands change:
+//   * a 128 x 128 tile is one 128-byte swizzle panel (16 KB);
 //   * tcgen05.mma kind::f8f6f4 consumes 32 elements of the reduction per
 //     instruction: S = Q K^T is 4 MMAs and O += P V is 4 MMAs per block, half
-//     the tensor-core time of bf16, which leaves the exponentials as the bound;
+//     the tensor-core time of bf16, which leaves the softmax as the bound;
+//   * so the softmax must never wait for the tensor core.  P (16 KB per tile
+//     in E4M3) goes to a double-buffered shared-memory tile instead of over S
+//     in TMEM, and a warp signals "S consumed" as soon as its scores are in
+//     registers: the MMA warp then computes the next block's S while this
+//     block is exponentiated, and P V runs behind, off the softmax's path;
 //   * the softmax warps read S with the .16x32bx2 TMEM shape: thread t of a
 //     warp owns one row (lane t % 16 of the warp's 16 lanes) and 64
 //     consecutive keys (half t / 16 of the block).  Row reductions finish
-//     with one shuffle (lanes t and t ^ 16 share a row), and four consecutive
-//     keys of P pack into one 32-bit TMEM column, the A-operand layout of an
-//     8-bit MMA, without any exchange between threads;
-//   * P is rounded to E4M3, whose largest finite value is 448.  Blocks after
-//     the first exponentiate against the running max as it stands (as the
-//     bf16 kernel does) and redo the block against its exact max when a
-//     thread's share of a row sum passes 256, so every P stays below 448 and
-//     no value saturates.
+//     with one shuffle (lanes t and t ^ 16 share a row), and the thread's 64
+//     P bytes are four 16-byte chunks of the row of the K-major, 128-byte
+//     swizzled A operand;
+//   * P is rounded to E4M3, whose largest finite value is 448.  Every block's
+//     exact max is taken, but the running max m only moves to it when it
+//     exceeds m by more than 8 (log2 units): p = 2^(s - m) <= 2^8 = 256, so
+//     nothing saturates, and O and l are rescaled only on such rare jumps.
 //
-// TMEM columns (512): S_0/P_0 at 0, S_1/P_1 at 128, O_0 at 256, O_1 at 384;
-// P_t occupies the first 32 columns of S_t.  Head dim 128 only.
+// Shared memory: Q (2 x 16 KB), a ring of 8 K/V slots (16 KB each), P (2 tiles
+// x 2 buffers x 16 KB).  TMEM columns (512): S_0 at 0, S_1 at 128, O_0 at 256,
+// O_1 at 384.  Head dim 128 only.
 //
 // Every mbarrier wait is bounded (tc::wait_bar / tc::drain_bar); on expiry the
 // CTA records the timeout in the device status word, leaves its loops, drains
@@ -63,7 +67,7 @@ using tc::kUnitRows;
 
 constexpr int D = 128;                 // head dim (one 128-byte row of E4M3)
 constexpr int kSlots = 8;              // K/V ring slots
-constexpr float kP8Bound = 256.0f;     // largest share of a row sum accepted against a stale max
+constexpr float kMaxSlack = 8.0f;      // log2 units a block's max may exceed the running max by
 #ifndef FA_FP8_POLY_GROUPS
 #define FA_FP8_POLY_GROUPS 0
 #endif
@@ -77,15 +81,21 @@ struct Layout {
     static constexpr int kTileBytes = kBlockM * D;  // 128 rows x 128 one-byte elements
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = kQOff + 2 * kTileBytes;
-    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    // q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2],
-    // sched_full[kSchedDepth], sched_empty[kSchedDepth], drain
-    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1;
+    static constexpr int kPOff = kRingOff + kSlots * kTileBytes;  // P[tile][buffer]
+    static constexpr int kBarOff = kPOff + 4 * kTileBytes;
+    // mbarrier indices: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], s_free[2],
+    // p_full[2][2], p_free[2][2], o_full[2], sched_full[kSchedDepth], sched_empty[kSchedDepth], drain
+    static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarKvFull = 4, kBarKvEmpty = 4 + kSlots;
+    static constexpr int kBarSFull = 4 + 2 * kSlots, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2;
+    static constexpr int kBarPFree = kBarPFull + 4, kBarOFull = kBarPFree + 4, kBarSchedFull = kBarOFull + 2;
+    static constexpr int kBarSchedEmpty = kBarSchedFull + kSchedDepth, kBarDrain = kBarSchedEmpty + kSchedDepth;
+    static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag, unit ring
     static constexpr int kBytes = kMiscOff + 8 + 4 * kSchedDepth;
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
     static constexpr uint32_t kTmemO = 256;
+    static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
 struct Params {
@@ -193,6 +203,11 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, fl
     return r;
 }
 
+// Make this thread's shared-memory writes visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- kernel
 
 template <bool kCausal>
@@ -210,16 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
 
     const uint32_t bar0 = base + L::kBarOff;
-    auto q_full = [&](int t) { return bar0 + 8u * t; };
-    auto q_empty = [&](int t) { return bar0 + 8u * (2 + t); };
-    auto kv_full = [&](int s) { return bar0 + 8u * (4 + s); };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (4 + kSlots + s); };
-    auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * kSlots + t); };
-    auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * kSlots + t); };
-    auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * kSlots + t); };
-    auto sched_full = [&](int i) { return bar0 + 8u * (10 + 2 * kSlots + i); };
-    auto sched_empty = [&](int i) { return bar0 + 8u * (10 + 2 * kSlots + kSchedDepth + i); };
-    const uint32_t drain = bar0 + 8u * (10 + 2 * kSlots + 2 * kSchedDepth);
+    auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+    auto q_full = [&](int t) { return bar(L::kBarQFull + t); };
+    auto q_empty = [&](int t) { return bar(L::kBarQEmpty + t); };
+    auto kv_full = [&](int s) { return bar(L::kBarKvFull + s); };
+    auto kv_empty = [&](int s) { return bar(L::kBarKvEmpty + s); };
+    auto s_full = [&](int t) { return bar(L::kBarSFull + t); };
+    auto s_free = [&](int t) { return bar(L::kBarSFree + t); };
+    // P_t of block k is announced on p_full(t, k & 1): with the next S issued
+    // early, a tile's softmax can finish block k + 1 before the MMA warp has
+    // seen block k, so one barrier could complete two phases unobserved.
+    auto p_full = [&](int t, int b) { return bar(L::kBarPFull + 2 * t + b); };
+    auto p_free = [&](int t, int b) { return bar(L::kBarPFree + 2 * t + b); };
+    auto o_full = [&](int t) { return bar(L::kBarOFull + t); };
+    auto sched_full = [&](int i) { return bar(L::kBarSchedFull + i); };
+    auto sched_empty = [&](int i) { return bar(L::kBarSchedEmpty + i); };
+    const uint32_t drain = bar(L::kBarDrain);
 
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -231,7 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(q_full(t), 1);
             ptx::mbar_init(q_empty(t), 1);
             ptx::mbar_init(s_full(t), 1);
-            ptx::mbar_init(p_full(t), 32 * (kSoftmaxWarps / 2));
+            ptx::mbar_init(s_free(t), 32 * (kSoftmaxWarps / 2));
+            ptx::mbar_init(p_full(t, 0), 32 * (kSoftmaxWarps / 2));
+            ptx::mbar_init(p_full(t, 1), 32 * (kSoftmaxWarps / 2));
+            ptx::mbar_init(p_free(t, 0), 1);
+            ptx::mbar_init(p_free(t, 1), 1);
             ptx::mbar_init(o_full(t), 1);
         }
         for (int s = 0; s < kSlots; ++s) {
@@ -331,15 +356,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
+        // The whole warp runs the loop (warp-uniform descriptors and waits);
+        // one elected lane issues every MMA and commit.  Per block j and tile
+        // t: S_t(j+1) as soon as the softmax has read S_t(j), then P_t(j) V_j
+        // as soon as P_t(j) is in shared memory.
         const bool leader = ptx::elect_one();
         constexpr uint32_t idesc_s = make_idesc_e4m3(kBlockM, kBlockN, false);
         constexpr uint32_t idesc_o = make_idesc_e4m3(kBlockM, D, true);
         const uint64_t desc_q0 = ptx::make_smem_desc(base + L::kQOff, 16, 1024);
         const uint64_t desc_k0 = ptx::make_smem_desc(base + L::kRingOff, 16, 1024);
         const uint64_t desc_v0 = ptx::make_smem_desc(base + L::kRingOff, L::kTileBytes, 1024);
+        const uint64_t desc_p0 = ptx::make_smem_desc(base + L::kPOff, 16, 1024);
         int slot = 0;
         uint32_t phase = 0;
-        uint32_t p_phase[2] = {0, 0};
+        uint32_t sf_phase[2] = {0, 0};
+        uint32_t pv_count[2] = {0, 0};  // P V products issued per tile (selects the P buffer)
         bool ok = true;
 
         // S_t = Q_t K^T: 4 MMAs of 32 elements (32 bytes along the swizzled row).
@@ -350,16 +381,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = 0; ks < D / 32; ++ks)
                 if (leader) mma_ss_f8(tmem + L::kTmemS + t * kBlockN, qd + 2 * ks, kd + 2 * ks, idesc_s, ks > 0);
         };
-        // O_t (+)= P_t V: 4 MMAs of 32 keys; P from TMEM (8 columns per 32
-        // keys), V from shared memory as an MN-major operand (32 rows of
-        // 128 bytes per step).
+        // O_t (+)= P_t V: 4 MMAs of 32 keys; P from its shared-memory buffer
+        // (K-major like Q), V as an MN-major operand (32 rows of 128 bytes per step).
         auto issue_pv = [&](int t, int vslot, bool accumulate) {
+            const int b = static_cast<int>(pv_count[t] & 1u);
+            const uint64_t pd = desc_p0 + (((2 * t + b) * L::kTileBytes) >> 4);
             const uint64_t vd = desc_v0 + ((vslot * L::kTileBytes) >> 4);
 #pragma unroll
             for (int ks = 0; ks < kBlockN / 32; ++ks)
                 if (leader)
-                    mma_ts_f8(tmem + L::kTmemO + t * D, tmem + L::kTmemS + t * kBlockN + ks * 8,
-                              vd + ((ks * 32 * 128) >> 4), idesc_o, (accumulate || ks > 0) ? 1u : 0u);
+                    mma_ss_f8(tmem + L::kTmemO + t * D, pd + 2 * ks, vd + ((ks * 32 * 128) >> 4), idesc_o,
+                              (accumulate || ks > 0) ? 1u : 0u);
+            if (leader) ptx::mma_commit(p_free(t, b));  // the buffer may be rewritten once these complete
+            ++pv_count[t];
         };
         auto commit = [&](uint32_t bar) {
             if (leader) ptx::mma_commit(bar);
@@ -405,41 +439,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             commit(kv_empty(sk));
 
             for (int j = 0; j < n1 && ok; ++j) {
-                next_slot(sv, pv);
-                ok = wait_all(kv_full(sv), pv);
-                if (!ok) break;
-                const bool more = j + 1 < n1;
-                if (more) {
+                const bool more0 = j + 1 < n0, more1 = j + 1 < n1;
+                next_slot(sv, pv);  // V_j (loaded before K_{j+1})
+                if (more1) {
                     next_slot(sk, pk);
                     ok = wait_all(kv_full(sk), pk);
                     if (!ok) break;
                 }
-                if (j < n0) {
-                    ok = wait_all(p_full(0), p_phase[0]);
+                if (more0) {
+                    ok = wait_all(s_free(0), sf_phase[0]);
                     if (!ok) break;
-                    p_phase[0] ^= 1;
+                    sf_phase[0] ^= 1;
                     ptx::tc_fence_after_sync();
-                    issue_pv(0, sv, j > 0);
-                    if (j == n0 - 1) commit(o_full(0));
-                }
-                if (j + 1 < n0) {
                     issue_s(0, sk);
                     commit(s_full(0));
                     if (j + 1 == n0 - 1) commit(q_empty(0));
                 }
-                ok = wait_all(p_full(1), p_phase[1]);
-                if (!ok) break;
-                p_phase[1] ^= 1;
-                ptx::tc_fence_after_sync();
-                issue_pv(1, sv, j > 0);
-                if (j == n1 - 1) commit(o_full(1));
-                commit(kv_empty(sv));
-                if (more) {
+                if (more1) {
+                    ok = wait_all(s_free(1), sf_phase[1]);
+                    if (!ok) break;
+                    sf_phase[1] ^= 1;
+                    ptx::tc_fence_after_sync();
                     issue_s(1, sk);
                     commit(s_full(1));
                     if (j + 1 == n1 - 1) commit(q_empty(1));
                     commit(kv_empty(sk));
                 }
+                ok = wait_all(kv_full(sv), pv);
+                if (!ok) break;
+                if (j < n0) {
+                    ok = wait_all(p_full(0, pv_count[0] & 1u), (pv_count[0] >> 1) & 1u);
+                    if (!ok) break;
+                    ptx::tc_fence_after_sync();
+                    issue_pv(0, sv, j > 0);
+                    if (j == n0 - 1) commit(o_full(0));
+                }
+                ok = wait_all(p_full(1, pv_count[1] & 1u), (pv_count[1] >> 1) & 1u);
+                if (!ok) break;
+                ptx::tc_fence_after_sync();
+                issue_pv(1, sv, j > 0);
+                if (j == n1 - 1) commit(o_full(1));
+                commit(kv_empty(sv));
             }
         }
         commit(drain);
@@ -459,8 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q + 16 * h) << 16;
         const uint32_t tmem_s = tmem + lane_addr + L::kTmemS + t * kBlockN;
         const uint32_t tmem_o = tmem + lane_addr + L::kTmemO + t * D;
+        // This thread's 64 bytes of a P row: chunks 4 c2 .. 4 c2 + 3 (16 bytes
+        // each) of row rr, placed by the 128-byte swizzle (chunk ^ row % 8).
+        uint8_t* p_row = smem + L::kPOff + t * 2 * L::kTileBytes + (rr >> 3) * 1024 + (rr & 7) * 128;
         const float sl = p.scale_log2;
         uint32_t s_phase = 0, o_phase = 0;
+        uint32_t blk = 0;  // blocks this thread has processed (P buffer blk & 1)
         bool ok = true;
 
         for (uint32_t it = 0; ok; ++it) {
@@ -479,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_run = -INFINITY;  // running max of the row, log2 units
             float l_run = 0.f;        // this thread's share of the row sum
 
-            for (int j = 0; j < nt; ++j) {
+            for (int j = 0; j < nt; ++j, ++blk) {
                 ok = __all_sync(0xffffffffu, tc::wait_bar(sync, s_full(t), s_phase));
                 if (!ok) break;
                 s_phase ^= 1;
@@ -491,101 +535,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float slv = need_mask ? 1.f : sl;  // masked blocks are pre-scaled
                 uint32_t sr[64];
                 float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
-                auto load_scores = [&]() {
-                    tmem_ld16x32bx2_x64_wait<64>(tmem_s, sr);
-                    if (need_mask) {
-                        const int lim = kCausal ? min(p.n - 1, row) : (p.n - 1);
+                tmem_ld16x32bx2_x64_wait<64>(tmem_s, sr);
+                // S_t is in registers: the tensor core may overwrite it with
+                // the next block's scores while this one is exponentiated.
+                if (j + 1 < nt) {
+                    ptx::tc_fence_before_sync();
+                    ptx::mbar_arrive(s_free(t));
+                }
+                if (need_mask) {
+                    const int lim = kCausal ? min(p.n - 1, row) : (p.n - 1);
 #pragma unroll
-                        for (int i = 0; i < 64; ++i) s[i] = (key0 + i <= lim) ? s[i] * sl : -INFINITY;
-                    }
-                };
+                    for (int i = 0; i < 64; ++i) s[i] = (key0 + i <= lim) ? s[i] * sl : -INFINITY;
+                }
                 // Exact row max in log2 units (both halves of the row): four
                 // running extremes over s[0..59] in steps of eight, then s[60..63].
                 auto block_max = [&]() {
-                    float c0 = s[0], c1 = s[1], c2 = s[2], c3 = s[3];
+                    float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
                     if (slv >= 0.f) {
 #pragma unroll
                         for (int i = 4; i < 60; i += 8) {
-                            c0 = ptx::max3(c0, s[i], s[i + 1]);
-                            c1 = ptx::max3(c1, s[i + 2], s[i + 3]);
-                            c2 = ptx::max3(c2, s[i + 4], s[i + 5]);
-                            c3 = ptx::max3(c3, s[i + 6], s[i + 7]);
+                            e0 = ptx::max3(e0, s[i], s[i + 1]);
+                            e1 = ptx::max3(e1, s[i + 2], s[i + 3]);
+                            e2 = ptx::max3(e2, s[i + 4], s[i + 5]);
+                            e3 = ptx::max3(e3, s[i + 6], s[i + 7]);
                         }
-                        c0 = ptx::max3(c0, s[60], s[61]);
-                        c1 = ptx::max3(c1, s[62], s[63]);
-                        float mx = fmaxf(fmaxf(c0, c1), fmaxf(c2, c3));
+                        e0 = ptx::max3(e0, s[60], s[61]);
+                        e1 = ptx::max3(e1, s[62], s[63]);
+                        float mx = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                         return mx * slv;
                     }
 #pragma unroll
                     for (int i = 4; i < 60; i += 8) {
-                        c0 = ptx::min3(c0, s[i], s[i + 1]);
-                        c1 = ptx::min3(c1, s[i + 2], s[i + 3]);
-                        c2 = ptx::min3(c2, s[i + 4], s[i + 5]);
-                        c3 = ptx::min3(c3, s[i + 6], s[i + 7]);
+                        e0 = ptx::min3(e0, s[i], s[i + 1]);
+                        e1 = ptx::min3(e1, s[i + 2], s[i + 3]);
+                        e2 = ptx::min3(e2, s[i + 4], s[i + 5]);
+                        e3 = ptx::min3(e3, s[i + 6], s[i + 7]);
                     }
-                    c0 = ptx::min3(c0, s[60], s[61]);
-                    c1 = ptx::min3(c1, s[62], s[63]);
-                    float mn = fminf(fminf(c0, c1), fminf(c2, c3));
+                    e0 = ptx::min3(e0, s[60], s[61]);
+                    e1 = ptx::min3(e1, s[62], s[63]);
+                    float mn = fminf(fminf(e0, e1), fminf(e2, e3));
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 16));
                     return mn * slv;
                 };
                 // p = 2^(s * slv - m), packed four keys per 32-bit word (the
-                // first key in the low byte), and this thread's share of the
-                // row sum over the unrounded values.
-                uint32_t pk[16];
+                // first key in the low byte) and written as four 16-byte
+                // chunks of the row to P buffer `prow`; a0 + a1 is this
+                // thread's share of the row sum over the unrounded values.
                 float a0, a1;
-                auto exponentiate = [&](float neg_m) {
+                auto exponentiate = [&](float neg_m, uint8_t* prow) {
                     a0 = a1 = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float x0, x1, x2, x3;
-                        ptx::fma2(x0, x1, s[4 * i], s[4 * i + 1], slv, slv, neg_m, neg_m);
-                        ptx::fma2(x2, x3, s[4 * i + 2], s[4 * i + 3], slv, slv, neg_m, neg_m);
-                        float p0, p1, p2, p3;
-                        if (!need_mask && i * kPolyGroups % 16 < kPolyGroups) {
-                            ptx::exp2_poly2(p0, p1, x0, x1);
-                            ptx::exp2_poly2(p2, p3, x2, x3);
-                        } else {
-                            p0 = ptx::ex2(x0);
-                            p1 = ptx::ex2(x1);
-                            p2 = ptx::ex2(x2);
-                            p3 = ptx::ex2(x3);
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t wd[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int i = 4 * c + k;
+                            float x0, x1, x2, x3;
+                            ptx::fma2(x0, x1, s[4 * i], s[4 * i + 1], slv, slv, neg_m, neg_m);
+                            ptx::fma2(x2, x3, s[4 * i + 2], s[4 * i + 3], slv, slv, neg_m, neg_m);
+                            float p0, p1, p2, p3;
+                            if (!need_mask && i * kPolyGroups % 16 < kPolyGroups) {
+                                ptx::exp2_poly2(p0, p1, x0, x1);
+                                ptx::exp2_poly2(p2, p3, x2, x3);
+                            } else {
+                                p0 = ptx::ex2(x0);
+                                p1 = ptx::ex2(x1);
+                                p2 = ptx::ex2(x2);
+                                p3 = ptx::ex2(x3);
+                            }
+                            wd[k] = pack_e4m3x4(p0, p1, p2, p3);
+                            ptx::add2(a0, a1, a0, a1, p0, p1);
+                            ptx::add2(a0, a1, a0, a1, p2, p3);
                         }
-                        pk[i] = pack_e4m3x4(p0, p1, p2, p3);
-                        ptx::add2(a0, a1, a0, a1, p0, p1);
-                        ptx::add2(a0, a1, a0, a1, p2, p3);
+                        const int chunk = (4 * c2 + c) ^ (rr & 7);
+                        *reinterpret_cast<uint4*>(prow + 16 * chunk) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
                     }
                 };
                 auto neg_of = [](float m) { return (m == -INFINITY) ? 0.f : -m; };
 
-                // Online softmax with a stale running max (see the file
-                // header): a block is redone against its exact max when a
-                // thread's share of the row sum passes kP8Bound.
-                load_scores();
+                // Online softmax with a lazily moved running max (see the file
+                // header): m moves to the block's max only when that exceeds
+                // it by more than kMaxSlack, so every p stays <= 2^kMaxSlack.
                 float alpha = 1.f;
                 bool rescale_o = false;
+                const float mx = block_max();
                 if (j == 0) {
-                    m_run = block_max();
-                    exponentiate(neg_of(m_run));
-                } else {
-                    exponentiate(neg_of(m_run));
-                    if (__any_sync(0xffffffffu, a0 + a1 > kP8Bound)) {
-                        load_scores();  // P has not been stored: S is still in TMEM
-                        const float mx = block_max();
-                        if (mx > m_run) {
-                            alpha = ptx::ex2(m_run - mx);
-                            m_run = mx;
-                            rescale_o = true;
-                        }
-                        exponentiate(neg_of(m_run));
-                    }
+                    m_run = mx;
+                } else if (mx > m_run + kMaxSlack) {
+                    alpha = ptx::ex2(m_run - mx);
+                    m_run = mx;
+                    rescale_o = true;
                 }
+                // P_t(j) goes to buffer blk & 1 once the P V that read it two
+                // blocks ago is complete.
+                const int b = static_cast<int>(blk & 1u);
+                if (blk >= 2) {
+                    ok = __all_sync(0xffffffffu, tc::wait_bar(sync, p_free(t, b), ((blk >> 1) - 1) & 1u));
+                    if (!ok) break;
+                }
+                exponentiate(neg_of(m_run), p_row + b * L::kTileBytes);
                 l_run = l_run * alpha + (a0 + a1);
-                tmem_st16x32bx2_x16<16>(tmem_s, pk);
 
-                // Rescale this row of O_t (both halves of the row agree on alpha).
+                // Rescale this row of O_t once P_t(j-1) V is complete (both
+                // halves of the row agree on alpha).
                 if (__any_sync(0xffffffffu, rescale_o)) {
+                    const uint32_t prev = blk - 1;
+                    ok = __all_sync(0xffffffffu,
+                                    tc::wait_bar(sync, p_free(t, static_cast<int>(prev & 1u)), (prev >> 1) & 1u));
+                    if (!ok) break;
+                    ptx::tc_fence_after_sync();
 #pragma unroll
                     for (int c0 = 0; c0 < D / 2; c0 += 16) {
                         uint32_t ov[16];
@@ -594,10 +653,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                         tmem_st16x32bx2_x16<64>(tmem_o + c0, ov);
                     }
+                    ptx::tmem_st_wait();
                 }
-                ptx::tmem_st_wait();
+                fence_async_shared();
                 ptx::tc_fence_before_sync();
-                ptx::mbar_arrive(p_full(t));
+                ptx::mbar_arrive(p_full(t, b));
             }
             if (!ok) break;
 
