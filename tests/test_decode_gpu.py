@@ -4,7 +4,10 @@ Element-by-element on every query, with the tolerances of the forward (bf16
 O 1e-2 max-abs and 1e-3 mean-abs, fp32 1e-5, lse 1e-3), over cache lengths
 that are not multiples of the 32-key tile, a single cached key, one to 13
 queries (two query groups), causal and not, heads split into many chunks
-(partials merged by the last CTA) and heads kept whole."""
+(partials merged by the last CTA) and heads kept whole.  One query per head
+runs on CUDA cores; 2 to 16 (bf16) on the warp-level MMA kernel, whose cases
+include a full 16-query group, a 17th query in a second group and caches
+shorter than one 32-key tile."""
 import math
 
 import numpy as np
@@ -52,6 +55,12 @@ CASES = [
     (4, 8, 1, 33, 64, False),
     (1, 2, 3, 4099, 64, True),
     (3, 1, 1, 65_536, 64, True),
+    # several queries run on the warp MMA in groups of 16 (bf16)
+    (1, 2, 2, 300, 64, True),
+    (2, 3, 16, 4000, 128, True),     # exactly one full group
+    (1, 2, 17, 3000, 128, True),     # a second group of one query
+    (1, 1, 16, 70_000, 64, False),   # one group, many chunks
+    (2, 2, 5, 31, 128, False),       # fewer keys than one tile
 ]
 
 
@@ -74,10 +83,11 @@ def test_decode_fp32_matches_oracle(B, H, nq, nk, d, causal):
     compare(o, lse, o_ref, lse_ref, torch.float32)
 
 
-def test_decode_wide_scores():
+@pytest.mark.parametrize("nq", [1, 2, 12])
+def test_decode_wide_scores(nq):
     # queries scaled by 8: scores spread over ~100 natural-log units, so the
     # running max moves often and chunk partials differ by huge factors
-    q, k, v = make(1, 4, 2, 20_000, 128, torch.bfloat16, seed=5, q_mult=8.0)
+    q, k, v = make(1, 4, nq, 20_000, 128, torch.bfloat16, seed=5, q_mult=8.0)
     o, lse = run(q, k, v, 1.0 / math.sqrt(128), True)
     o_ref, lse_ref = reference(q, k, v, 1.0 / math.sqrt(128), True)
     compare(o, lse, o_ref, lse_ref, torch.bfloat16, strict_raw=False)

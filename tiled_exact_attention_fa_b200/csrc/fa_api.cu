@@ -19,6 +19,7 @@
 #include "fa_testing.h"
 #include "fa_bwd_tc.cuh"
 #include "fa_decode.cuh"
+#include "fa_decode_mma.cuh"
 #include "fa_merge.cuh"
 #include "fa_fwd_fp8_tc.cuh"
 #include "fa_fwd_simt.cuh"
@@ -61,6 +62,7 @@ struct DeviceState {
     bool decode_smem_raised[8] = {false, false, false, false, false, false, false, false};
     bool bwd_smem_raised[8] = {false, false, false, false, false, false, false, false};
     bool fp8_smem_raised[2] = {false, false};
+    bool decode_mma_smem_raised[2] = {false, false};
 };
 
 constexpr int kMaxDevices = 64;
@@ -106,12 +108,13 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-// 3-D view (d, N, B*H) of a [B*H][N][d] bf16 tensor, boxes of 64 x 128 x 1
-// with 128-byte swizzle; rows past N read as zeros.
-int encode_tile_map(CUtensorMap* map, const void* ptr, int64_t bh, int64_t n, int64_t d) {
+// 3-D view (d, N, B*H) of a [B*H][N][d] bf16 tensor, boxes of 64 x rows x 1
+// (rows = 128 unless given) with 128-byte swizzle; rows past N read as zeros.
+int encode_tile_map(CUtensorMap* map, const void* ptr, int64_t bh, int64_t n, int64_t d,
+                    int rows = fa::tc::kBlockM) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(bh)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(n * d * 2)};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fa::tc::kBlockM), 1};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
     cuuint32_t elem[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -610,10 +613,17 @@ struct DecodePlan {
     size_t part_bytes = 0, count_bytes = 0, workspace = 0;
 };
 
-DecodePlan decode_plan(int64_t bh, int64_t nq, int64_t nk, int64_t d) {
+// Queries per CTA: one at a time on CUDA cores; groups of 16 on the warp MMA
+// (bf16) or of 4 on CUDA cores (fp32).
+int64_t decode_tile(int64_t nq, int dtype) {
+    if (nq == 1) return 1;
+    return dtype == FA_DTYPE_BF16 ? fa::decm::kQ : fa::dec::kMaxQ;
+}
+
+DecodePlan decode_plan(int64_t bh, int64_t nq, int64_t nk, int64_t d, int64_t nq_tile) {
     DecodePlan pl;
     pl.bh = bh;
-    pl.nq_tile = nq == 1 ? 1 : fa::dec::kMaxQ;
+    pl.nq_tile = nq_tile;
     pl.groups = (nq + pl.nq_tile - 1) / pl.nq_tile;
     const int64_t ctas = bh * pl.groups;
     int64_t chunks = (kDecodeTargetCtas + ctas - 1) / ctas;
@@ -645,7 +655,7 @@ int decode_check(const void* q, const void* k, const void* v, const void* o, con
     if (B > (int64_t{1} << 24) / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
     const int64_t bh = B * H;
     const int64_t elem = dtype == FA_DTYPE_BF16 ? 2 : 4;
-    *pl = decode_plan(bh, Nq, Nk, d);
+    *pl = decode_plan(bh, Nq, Nk, d, decode_tile(Nq, dtype));
     if (pl->groups > 65535) return fail(FA_ERR_INVALID_ARGUMENT, "too many query groups");
     if (bh * pl->chunks > INT_MAX) return fail(FA_ERR_INVALID_ARGUMENT, "B * H * chunks too large");
     auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
@@ -678,11 +688,36 @@ int launch_decode(DeviceState* st, int slot, const fa::dec::Params& p, const Dec
     return FA_OK;
 }
 
+template <int D>
+int launch_decode_mma(DeviceState* st, int slot, const fa::dec::Params& p, const DecodePlan& pl, cudaStream_t s) {
+    using C = fa::decm::Cfg<D>;
+    auto kernel = fa::decm::fa_decode_mma_kernel<D>;
+    if (!st->decode_mma_smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->decode_mma_smem_raised[slot] = true;
+    }
+    CUtensorMap tk, tv;
+    int rc;
+    if ((rc = encode_tile_map(&tk, p.k, pl.bh, p.nk, D, fa::dec::kTileKeys)) != FA_OK ||
+        (rc = encode_tile_map(&tv, p.v, pl.bh, p.nk, D, fa::dec::kTileKeys)) != FA_OK)
+        return rc;
+    dim3 grid(static_cast<unsigned>(pl.bh * pl.chunks), static_cast<unsigned>(pl.groups));
+    kernel<<<grid, fa::dec::kThreads, C::kSmemBytes, s>>>(tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the decode (warp MMA) kernel");
+    return FA_OK;
+}
+
 }  // namespace
 
+// The size covers either dtype's plan (the argument list has no dtype).
 extern "C" size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d) {
     if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || B > (int64_t{1} << 24) / H) return 0;
-    return decode_plan(B * H, Nq, Nk, d).workspace;
+    const size_t a = decode_plan(B * H, Nq, Nk, d, decode_tile(Nq, FA_DTYPE_BF16)).workspace;
+    const size_t b = decode_plan(B * H, Nq, Nk, d, decode_tile(Nq, FA_DTYPE_F32)).workspace;
+    return a > b ? a : b;
 }
 
 extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
@@ -724,6 +759,8 @@ extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, f
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode counters)");
     }
     const bool one = pl.nq_tile == 1;
+    if (dtype == FA_DTYPE_BF16 && pl.nq_tile == fa::decm::kQ)
+        return d == 128 ? launch_decode_mma<128>(st, 0, p, pl, s) : launch_decode_mma<64>(st, 1, p, pl, s);
     if (dtype == FA_DTYPE_BF16) {
         if (d == 128) return one ? launch_decode<__nv_bfloat16, 128, 1>(st, 0, p, pl, s)
                                  : launch_decode<__nv_bfloat16, 128, fa::dec::kMaxQ>(st, 1, p, pl, s);
