@@ -95,8 +95,10 @@ def traffic_from_profile(w):
         return None
     with open(path) as f:
         d = json.load(f)
-    kind = ("decode" if isinstance(w, W.DecodeWorkload) else
-            "forward_fp8" if w.dtype == torch.float8_e4m3fn else "forward")
+    if isinstance(w, W.DecodeWorkload):
+        kind = "decode_mma" if w.dtype == torch.bfloat16 else "decode"
+    else:
+        kind = "forward_fp8" if w.dtype == torch.float8_e4m3fn else "forward"
     if d.get("kernel_digest") != kernel_digest(kind):
         return None
     return d.get("dram_bytes_per_launch")
@@ -553,7 +555,8 @@ def run_decode(a, w: W.DecodeWorkload):
         line["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                             "peak_kind": f"{peak_kind} HBM copy bandwidth",
                             "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
-                            "kernel": f"fa_decode_kernel<{'bf16' if esz == 2 else 'f32'},{w.d},{1 if w.nq == 1 else 4}>"}
+                            "kernel": f"fa_decode_mma_kernel<{w.d}>" if esz == 2 else
+                            f"fa_decode_kernel<f32,{w.d},{1 if w.nq == 1 else 4}>"}
         line["clocks"] = clocks.summary()
         line["gpu_launches"] = a.steps
     if "e2e" in legs:

@@ -4,10 +4,10 @@ Element-by-element on every query, with the tolerances of the forward (bf16
 O 1e-2 max-abs and 1e-3 mean-abs, fp32 1e-5, lse 1e-3), over cache lengths
 that are not multiples of the 32-key tile, a single cached key, one to 13
 queries (two query groups), causal and not, heads split into many chunks
-(partials merged by the last CTA) and heads kept whole.  One query per head
-runs on CUDA cores; 2 to 16 (bf16) on the warp-level MMA kernel, whose cases
-include a full 16-query group, a 17th query in a second group and caches
-shorter than one 32-key tile."""
+(partials merged by the last CTA) and heads kept whole.  bf16 runs on the
+warp-level MMA kernel in groups of 16 queries (cases include a full group,
+a 17th query in a second group and caches shorter than one 32-key tile);
+fp32 on the CUDA-core kernel."""
 import math
 
 import numpy as np

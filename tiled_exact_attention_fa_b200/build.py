@@ -71,6 +71,7 @@ def code_digest(files=None) -> str:
 KERNEL_SOURCES = {
     "forward": ["fa_fwd_tc.cuh", "sm100_ptx.cuh"],
     "decode": ["fa_decode.cuh", "sm100_ptx.cuh"],
+    "decode_mma": ["fa_decode_mma.cuh", "fa_decode.cuh", "sm100_ptx.cuh"],
     "forward_fp8": ["fa_fwd_fp8_tc.cuh", "fa_fwd_tc.cuh", "sm100_ptx.cuh"],
 }
 

@@ -613,11 +613,12 @@ struct DecodePlan {
     size_t part_bytes = 0, count_bytes = 0, workspace = 0;
 };
 
-// Queries per CTA: one at a time on CUDA cores; groups of 16 on the warp MMA
-// (bf16) or of 4 on CUDA cores (fp32).
+// Queries per CTA: bf16 in groups of 16 on the warp MMA (one query too: the
+// padded tile's tensor work is still far below the loads, and the swizzled
+// tensor copies stream faster); fp32 on CUDA cores, one query or groups of 4.
 int64_t decode_tile(int64_t nq, int dtype) {
-    if (nq == 1) return 1;
-    return dtype == FA_DTYPE_BF16 ? fa::decm::kQ : fa::dec::kMaxQ;
+    if (dtype == FA_DTYPE_BF16) return fa::decm::kQ;
+    return nq == 1 ? 1 : fa::dec::kMaxQ;
 }
 
 DecodePlan decode_plan(int64_t bh, int64_t nq, int64_t nk, int64_t d, int64_t nq_tile) {
@@ -759,14 +760,8 @@ extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, f
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode counters)");
     }
     const bool one = pl.nq_tile == 1;
-    if (dtype == FA_DTYPE_BF16 && pl.nq_tile == fa::decm::kQ)
+    if (dtype == FA_DTYPE_BF16)
         return d == 128 ? launch_decode_mma<128>(st, 0, p, pl, s) : launch_decode_mma<64>(st, 1, p, pl, s);
-    if (dtype == FA_DTYPE_BF16) {
-        if (d == 128) return one ? launch_decode<__nv_bfloat16, 128, 1>(st, 0, p, pl, s)
-                                 : launch_decode<__nv_bfloat16, 128, fa::dec::kMaxQ>(st, 1, p, pl, s);
-        return one ? launch_decode<__nv_bfloat16, 64, 1>(st, 2, p, pl, s)
-                   : launch_decode<__nv_bfloat16, 64, fa::dec::kMaxQ>(st, 3, p, pl, s);
-    }
     if (d == 128) return one ? launch_decode<float, 128, 1>(st, 4, p, pl, s)
                              : launch_decode<float, 128, fa::dec::kMaxQ>(st, 5, p, pl, s);
     return one ? launch_decode<float, 64, 1>(st, 6, p, pl, s) : launch_decode<float, 64, fa::dec::kMaxQ>(st, 7, p, pl, s);

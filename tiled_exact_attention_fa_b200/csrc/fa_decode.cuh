@@ -1,4 +1,5 @@
-// fa_decode.cuh -- attention of a few new queries over a long key/value cache.
+// fa_decode.cuh -- attention of a few new queries over a long key/value cache
+// on CUDA cores (the fp32 path; bf16 runs on the warp MMA, fa_decode_mma.cuh).
 //
 // What it computes (per head): for nq new queries and nk cached keys (the
 // new tokens' own keys are the last nq of them), O = softmax(scale * Q K^T

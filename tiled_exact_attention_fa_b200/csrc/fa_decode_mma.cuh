@@ -1,10 +1,10 @@
-// fa_decode_mma.cuh -- attention of 2 to 16 new queries per head over a long
-// key/value cache, on the warp-level tensor-core MMA.
+// fa_decode_mma.cuh -- attention of new queries over a long key/value cache
+// (bf16), on the warp-level tensor-core MMA.
 //
 // Same operation, split-KV plan, workspace and merge as fa_decode.cuh
 // ("FlashAttention: Tiled & Fused", card "KV Cache: Why Generation Speeds
 // Up"; online softmax of "FlashAttention, Playable", EP 04).  What changes is
-// the arithmetic per key: with several queries the CUDA-core kernel spends
+// the arithmetic per key: with several queries a CUDA-core kernel spends
 // about 1000 multiply-adds and a dozen shuffles per key and query group and
 // runs out of issue slots below HBM speed.  Here a warp multiplies a 16-query
 // tile (the group, padded with zero rows) by 8 keys at a time:
@@ -14,8 +14,9 @@
 // first product is the A layout of the second once packed to bf16), K
 // fragments from ldmatrix and V fragments from ldmatrix.trans.  That is
 // about six warp instructions per key instead of fifty, so the kernel is
-// bound by HBM again.  The queries are padded 4x at nq = 4; the tensor work
-// is still far below what the loads take.
+// bound by HBM again.  Any number of queries runs in groups of 16 (a single
+// query too: padded 16x, the tensor work is still far below what the loads
+// take).
 //
 // Shared memory: a 4-stage ring of 32-key K and V tiles, each loaded by TMA
 // as d/64 panels of 32 rows x 128 bytes with the 128-byte swizzle (16-byte
