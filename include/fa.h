@@ -200,8 +200,10 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse
  *
  * The key range of each head is split into chunks that separate CTAs process
  * (partial results merged by their log-sum-exp, as the online softmax
- * merges tiles), so a single long head still uses the whole GPU.  Errors and
- * asynchrony as for fa_fwd.  Alignment: q, k, v, o 16 bytes, lse 4 bytes.
+ * merges tiles), so a single long head still uses the whole GPU.  bf16 runs
+ * on the warp-level tensor-core MMA in groups of 16 queries (P rounded to
+ * bf16 before P V, as in fa_fwd); fp32 on CUDA cores.  Errors and asynchrony
+ * as for fa_fwd.  Alignment: q, k, v, o 16 bytes, lse 4 bytes.
  */
 int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
               int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d,
@@ -209,9 +211,10 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * fa_decode_workspace_bytes -- the workspace fa_decode needs for these sizes
- * (0 when one CTA per head suffices, or for invalid sizes).  Depends only on
- * the arguments, not on the device.
+ * fa_decode_workspace_bytes -- the workspace fa_decode needs for these sizes,
+ * for either dtype (the two dtypes group queries differently; the larger
+ * need is returned).  0 when one CTA per head and query group suffices, or
+ * for invalid sizes.  Depends only on the arguments, not on the device.
  */
 size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t d);
 
