@@ -128,9 +128,9 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
  * with fp32 accumulation, P rounded to E4M3 (nearest) as the operand of P V,
  * the running max and sum in fp32.  Q8 K8^T is exact in fp32 up to the
  * accumulation order; the rounding of P is the one approximation, and each
- * element of O lies within 2^-4 * sum_j p_j |v_j| + 2^-10 * sum_j |v_j| / l
- * (+ the bf16 rounding of O) of the exact result, p_j the exact softmax
- * weights and l = exp(lse - max_j s_j).
+ * element of O lies within |descale_v| (2^-4 sum_j p_j |v8_j| + 2^-10
+ * sum_j |v8_j| / l) (+ the bf16 rounding of O) of the exact result, p_j the
+ * exact softmax weights and l = exp(lse - max_j s_j).
  *
  *   q, k, v  device, contiguous [B][H][N][d] one-byte E4M3.  16-byte aligned.
  *   o        device, [B][H][N][d] bf16, written once per row.  16-byte aligned.
