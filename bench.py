@@ -366,7 +366,7 @@ def run_fp8(a, w: W.Workload):
     rows = w.B * w.H * w.N
     in_bytes = 3 * rows * w.d
     out_bytes = 2 * rows * w.d + 4 * rows
-    alg_bytes = in_bytes + out_bytes
+    alg_bytes = accounting.algorithmic_bytes(w.B, w.H, w.N, w.d, 1, out_elem_bytes=2)
 
     def step():
         fa.forward_fp8_into(q, k, v, o, lse, scale=w.scale, causal=w.causal)

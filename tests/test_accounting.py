@@ -25,6 +25,13 @@ def test_headline_flops_and_bytes():
     assert accounting.algorithmic_bytes(2, 32, 8192, 128, 2) == 4 * 2 * 32 * 8192 * 128 * 2 + 2 * 32 * 8192 * 4
 
 
+def test_fp8_bytes():
+    # E4M3 B=2 H=32 N=8192 d=128: one-byte Q, K, V, bf16 O, fp32 lse
+    rows = 2 * 32 * 8192
+    assert accounting.algorithmic_bytes(2, 32, 8192, 128, 1, out_elem_bytes=2) == \
+        3 * rows * 128 + 2 * rows * 128 + 4 * rows == 337641472
+
+
 def test_roofline_min():
     assert accounting.roofline_flops(4, 989e12, 3.35e12) == 4 * 3.35e12
     assert accounting.roofline_flops(1000, 989e12, 3.35e12) == 989e12

@@ -18,9 +18,14 @@ def attention_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
     return f / 2 if causal else f
 
 
-def algorithmic_bytes(B: int, H: int, N: int, d: int, elem_bytes: int, lse_bytes: int = 4) -> int:
+def algorithmic_bytes(B: int, H: int, N: int, d: int, elem_bytes: int, lse_bytes: int = 4,
+                      out_elem_bytes: int | None = None) -> int:
+    """Q, K, V read once (elem_bytes each), O written once (out_elem_bytes,
+    default elem_bytes) and one lse per row.  The E4M3 forward reads one-byte
+    inputs and writes bf16: elem_bytes=1, out_elem_bytes=2."""
     rows = B * H * N
-    return 4 * rows * d * elem_bytes + rows * lse_bytes
+    out = elem_bytes if out_elem_bytes is None else out_elem_bytes
+    return 3 * rows * d * elem_bytes + rows * d * out + rows * lse_bytes
 
 
 def score_matrix_elements(N: int) -> int:
