@@ -17,8 +17,10 @@ deliberately slow plain definition) on a bounded sample of the same workload.
 
 `--path ring` measures the sequence-parallel forward (ring of K/V chunks,
 partial results merged by log-sum-exp): under torchrun the real ring over
-NCCL, each rank holding one chunk of one sequence (strong scaling); on one
+NCCL over the ranks of one sequence (strong scaling); on one
 GPU the same schedule emulated for --ring-chunks ranks, one after another.
+Each rank holds two chunks of the sequence (chunks r and 2P-1-r of 2P, the
+zig-zag layout that gives every rank the same causal work).
 `--path backward` measures fa_bwd (dq, dk, dv from the saved lse) on the same
 workload, counting the customary 2.5x the forward's FLOPs.  `--path fp8`
 measures fa_fwd_fp8 (E4M3 Q, K, V, bf16 O) on an E4M3 workload of the same
@@ -741,6 +743,17 @@ def run_backward(a, w: W.Workload):
 RING_METRIC = "sequence-parallel attention fwd TFLOPS (bf16, d=128, N=8K causal; chunks merged by log-sum-exp)"
 
 
+def ring_launches_per_rank(world: int, causal: bool) -> int:
+    """Kernels one rank launches per ring step: fa_fwd per call of the
+    schedule, then fa_merge per query chunk (once for the whole rows when no
+    chunk-sized call was made)."""
+    from tiled_exact_attention_fa_b200 import ring
+    sched = ring.ring_schedule(0, world, causal)
+    calls = sum(len(c) for _, _, c in sched)
+    chunked = any(qp != ring.ALL for _, _, cs in sched for qp, _, _ in cs)
+    return calls + (2 if chunked else 1)
+
+
 def run_ring(a, w: W.Workload):
     import tiled_exact_attention_fa_b200 as fa
     from tiled_exact_attention_fa_b200 import ring
@@ -754,11 +767,9 @@ def run_ring(a, w: W.Workload):
         fdist.init("nccl", timeout_s=300)
     q, k, v = (x.to(dev) for x in W.make_inputs(w))  # the whole sequence, same on every rank
     chunks = world if world > 1 else a.ring_chunks
-    if w.N % chunks:
-        raise SystemExit("the sequence must split into equal chunks")
-    n = w.N // chunks
-    sl = slice(rank * n, (rank + 1) * n)
-    ql, kl, vl = (t[:, :, sl].contiguous() for t in (q, k, v))
+    if w.N % (2 * chunks):
+        raise SystemExit("the sequence must split into 2 * ranks equal chunks")
+    ql, kl, vl = (ring.zigzag_shard(t, rank, world) for t in (q, k, v)) if world > 1 else (q, k, v)
     stream = torch.cuda.current_stream(dev)
     flops = accounting.attention_flops(w.B, w.H, w.N, w.d, w.causal)
 
@@ -789,15 +800,14 @@ def run_ring(a, w: W.Workload):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "seed": w.seed, "chunks": chunks,
-                       "mode": "ring over NCCL, one chunk per rank" if world > 1 else
-                       f"{chunks} ranks emulated one after another on one GPU",
+                       "mode": "ring over NCCL, zig-zag chunk pair per rank" if world > 1 else
+                       f"{chunks} ranks (zig-zag chunk pairs) emulated one after another on one GPU",
                        "flop_per_step": flops},
             "roofline": {"bound": "tensor", "achieved": tf / world, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / world / peak, "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
                          "traffic": None, "kernel": "fa_fwd_bf16_kernel per chunk pair + fa_merge_kernel"},
             "clocks": clocks.summary(),
-            "gpu_launches": a.steps * (chunks * (chunks + 1) // 2 + chunks if w.causal else chunks * chunks + chunks)
-            // (world if world > 1 else 1)}
+            "gpu_launches": a.steps * ring_launches_per_rank(chunks, w.causal) * (1 if world > 1 else chunks)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

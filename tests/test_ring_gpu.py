@@ -1,7 +1,7 @@
 """fa_merge and the sequence-parallel arithmetic on one GPU: the merge kernel
-against the oracle's merge, and the ring schedule emulated rank by rank
-(fa_fwd on each chunk pair, fa_merge per rank) against the fp64 oracle on the
-whole sequence."""
+against the oracle's merge, and the zig-zag ring schedule emulated rank by
+rank (fa_fwd on each chunk pair, fa_merge per query chunk) against the fp64
+oracle on the whole sequence, up to the eight ranks the ring bench uses."""
 import math
 
 import numpy as np
@@ -36,7 +36,7 @@ def test_merge_kernel_matches_oracle(dtype, d):
     assert torch.isinf(lse[500]).item() and lse[500].item() < 0 and (o[500] == 0).all().item()
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [2, 4, 8])
 @pytest.mark.parametrize("causal", [False, True])
 def test_emulated_ring_matches_oracle(world, causal):
     fa_build.build()
