@@ -101,18 +101,36 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *   - The first call on a device, with that device current, looks up the
  *     array's device address (cudaGetSymbolAddress); make that first call
  *     before any stream capture.
- *   - Each call clears the array's status and queue words on `stream` before
- *     its kernel runs.  All calls share the one array: calls whose kernels can
+ *   - Each call clears the array's work-queue words on `stream` before its
+ *     kernel runs.  All calls share the one array: calls whose kernels can
  *     overlap on the GPU (different streams, several host threads) race on it
  *     and give wrong results; issue them in order on one stream.
- *   - A call that would need more scratch than the array holds is rejected
- *     with FA_ERR_UNSUPPORTED (the current kernels need 24 bytes).
- *   - A device-side timeout of a call made here is recorded only in the array,
- *     not reported by fa_check_device_status.
+ *   - The kernels use 24 of the array's 256 bytes (a compile-time check keeps
+ *     them inside it); no argument makes a call need more.
+ *   - A device-side timeout of a call made here (a bounded wait that ran out;
+ *     that call's o and lse are invalid) sets the array's status word, which
+ *     later calls leave set: fa_noalloc_check_status (below) reports it as
+ *     FA_ERR_DEVICE_TIMEOUT and clears it.  fa_check_device_status reads
+ *     fa_fwd's own status word, not this one.
+ *   - fp32 inputs run the fp32 kernel, which needs no scratch.
  */
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                    int64_t B, int64_t H, int64_t N, int64_t d,
                    float scale, int causal, int dtype, void* stream);
+
+/*
+ * fa_noalloc_check_status -- the status of the fa_fwd_noalloc calls made on
+ * the current device since the last check.  No counterpart in the pages (it
+ * belongs to the no-allocation variant above).  Synchronises `stream` (a
+ * cudaStream_t), reads the no-alloc array's status word with a plain
+ * device-to-host copy (nothing is allocated) and, if a kernel gave up on a
+ * bounded wait, clears the word and returns FA_ERR_DEVICE_TIMEOUT (the outputs
+ * of the call that timed out are invalid; the context stays usable).
+ * Returns FA_OK when no timeout was recorded, FA_ERR_CUDA if a CUDA call
+ * failed.  Like the calls it checks, it must not overlap another no-alloc
+ * call on the GPU.
+ */
+int fa_noalloc_check_status(void* stream);
 
 /*
  * fa_fwd_fp8 -- the attention forward with 8-bit float inputs.

@@ -27,10 +27,11 @@ extern "C" {
 int fa_test_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /*
- * fa_test_skip_one_arrival -- the next bf16 launch of fa_fwd in this process
- * runs with one arrival missing: CTA 0 never loads its first Q tile, so the
+ * fa_test_skip_one_arrival -- the next bf16 forward launch in this process
+ * (through fa_fwd or fa_fwd_noalloc) runs with one arrival missing: CTA 0 never loads its first Q tile, so the
  * MMA warp's bounded wait on that tile runs out (about two seconds).  The
- * kernel then records FA_ERR_DEVICE_TIMEOUT in the device status word,
+ * kernel then records FA_ERR_DEVICE_TIMEOUT in the status word of the entry
+ * point that launched it,
  * drains its copies and MMAs, frees its tensor memory and exits; the context
  * stays usable.  Exercises the failure-detection path of the bounded waits
  * (the pages have no counterpart).  Always returns FA_OK.

@@ -66,8 +66,8 @@ NB = 1 << 24  # spacing between the fake buffers
 
 
 def call(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,
-         scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16):
-    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, None)
+         scale=0.1, causal=0, dtype=fa.FA_DTYPE_BF16, entry="fa_fwd"):
+    return getattr(lib, entry)(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, None)
 
 
 @pytest.mark.parametrize("kwargs,code", [
@@ -93,9 +93,10 @@ def call(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=
     (dict(d=96), fa.FA_ERR_UNSUPPORTED),
     (dict(d=256), fa.FA_ERR_UNSUPPORTED),
 ])
-def test_rejected_before_cuda(lib, kwargs, code):
-    lib.fa_fwd.restype = ctypes.c_int
-    assert call(lib, **kwargs) == code
+@pytest.mark.parametrize("entry", ["fa_fwd", "fa_fwd_noalloc"])
+def test_rejected_before_cuda(lib, kwargs, code, entry):
+    # fa_fwd_noalloc runs the same checks, also before any CUDA call
+    assert call(lib, entry=entry, **kwargs) == code
     assert lib.fa_last_error().decode() != ""
 
 
@@ -103,6 +104,8 @@ def test_rejected_before_cuda(lib, kwargs, code):
 def test_no_gpu_is_an_error_not_a_fallback(lib):
     # well-formed arguments on a machine without a GPU: a CUDA error, never a result
     assert call(lib) == fa.FA_ERR_CUDA
+    assert call(lib, entry="fa_fwd_noalloc") == fa.FA_ERR_CUDA
+    assert lib.fa_noalloc_check_status(None) == fa.FA_ERR_CUDA
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises((RuntimeError, AssertionError)):
         fa.forward(q, q, q)

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "fa_merge": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fa_noalloc_check_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_version": (ctypes.c_int, []),

@@ -325,15 +325,17 @@ int fa_check_device_status(void* stream) {
 namespace {
 
 // 256 bytes of scratch, loaded with the library on every GPU it runs on and
-// kept until the process exits.  Word 0: device status (a kernel that gave up
-// on a bounded wait sets it); words 4 and 5: the persistent kernel's work
-// queue (next unit, CTAs finished).  The rest is unused headroom.
+// kept until the process exits (zero when the library is loaded).  Word 0:
+// device status (a kernel that gave up on a bounded wait sets it; it stays set
+// until fa_noalloc_check_status reads it); words 4 and 5: the persistent
+// kernel's work queue (next unit, CTAs finished), cleared before every launch.
+// The rest is unused headroom.
 constexpr int kNoAllocScratchWords = 64;
 constexpr int kNoAllocStatusWord = 0;
 constexpr int kNoAllocQueueWord = 4;
-constexpr int kNoAllocWordsUsed = 6;
+constexpr int kNoAllocQueueWords = 2;
 static __device__ __align__(256) unsigned g_noalloc_scratch[kNoAllocScratchWords];
-static_assert(kNoAllocWordsUsed <= kNoAllocScratchWords, "no-alloc scratch too small");
+static_assert(kNoAllocQueueWord + kNoAllocQueueWords <= kNoAllocScratchWords, "no-alloc scratch too small");
 
 struct NoAllocDevice {
     bool ready = false;
@@ -392,10 +394,11 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
-    // The array keeps the previous call's contents: the status word and the
-    // queue counters must start at zero, so clear them in stream order.
-    cudaError_t e = cudaMemsetAsync(st->scratch, 0, kNoAllocWordsUsed * sizeof(unsigned), stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc scratch)");
+    // The array keeps the previous call's contents: the queue counters must
+    // start at zero, so clear them in stream order.  The status word is left
+    // alone, so that a timeout stays visible until fa_noalloc_check_status.
+    cudaError_t e = cudaMemsetAsync(st->scratch + kNoAllocQueueWord, 0, kNoAllocQueueWords * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc queue words)");
 
     fa::tc::Params p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -408,7 +411,7 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
     p.num_units = p.bh * p.num_qblocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    p.skip_one_arrival = 0;
+    p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
     kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
@@ -447,9 +450,6 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
     if (overlaps(lse, lse_bytes, q, tensor_bytes) || overlaps(lse, lse_bytes, k, tensor_bytes) ||
         overlaps(lse, lse_bytes, v, tensor_bytes))
         return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
-    // the scratch this call needs must fit the fixed array
-    if (static_cast<size_t>(kNoAllocWordsUsed) * sizeof(unsigned) > sizeof(g_noalloc_scratch))
-        return fail(FA_ERR_UNSUPPORTED, "call needs more scratch than the 256-byte no-alloc array holds");
 
     // ---- set-up on the first call per device (no allocation) and dispatch
     NoAllocDevice* st = nullptr;
@@ -470,6 +470,24 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
                            : launch_f32<128, false>(q, k, v, o, lse, bh, N, scale, s);
     return c ? launch_f32<64, true>(q, k, v, o, lse, bh, N, scale, s)
              : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
+}
+
+extern "C" int fa_noalloc_check_status(void* stream) {
+    g_last_error.clear();
+    NoAllocDevice* st = nullptr;
+    int rc = noalloc_setup(&st);
+    if (rc != FA_OK) return rc;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned h = 0;
+    if ((e = cudaMemcpy(&h, st->scratch + kNoAllocStatusWord, sizeof(unsigned), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpy(no-alloc status word)");
+    if (h != 0) {
+        if ((e = cudaMemset(st->scratch + kNoAllocStatusWord, 0, sizeof(unsigned))) != cudaSuccess)
+            return cuda_fail(e, "cudaMemset(no-alloc status word)");
+        return fail(FA_ERR_DEVICE_TIMEOUT, "a kernel launched by fa_fwd_noalloc gave up on a bounded wait");
+    }
+    return FA_OK;
 }
 
 // ---------------------------------------------------------------------------

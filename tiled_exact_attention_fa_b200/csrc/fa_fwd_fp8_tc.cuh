@@ -68,14 +68,6 @@ using tc::kUnitRows;
 constexpr int D = 128;                 // head dim (one 128-byte row of E4M3)
 constexpr int kSlots = 8;              // K/V ring slots
 constexpr float kMaxSlack = 8.0f;      // log2 units a block's max may exceed the running max by
-#ifndef FA_FP8_POLY_GROUPS
-#define FA_FP8_POLY_GROUPS 0
-#endif
-// Of a thread's 16 groups of four scores per block, this many are
-// exponentiated on the FMA pipe (ptx::exp2_poly2) instead of the MUFU
-// (unmasked blocks only; the polynomial's 2^-13.7 relative error is far
-// below E4M3's 2^-4).
-constexpr int kPolyGroups = FA_FP8_POLY_GROUPS;
 
 struct Layout {
     static constexpr int kTileBytes = kBlockM * D;  // 128 rows x 128 one-byte elements
@@ -594,16 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float x0, x1, x2, x3;
                             ptx::fma2(x0, x1, s[4 * i], s[4 * i + 1], slv, slv, neg_m, neg_m);
                             ptx::fma2(x2, x3, s[4 * i + 2], s[4 * i + 3], slv, slv, neg_m, neg_m);
-                            float p0, p1, p2, p3;
-                            if (!need_mask && i * kPolyGroups % 16 < kPolyGroups) {
-                                ptx::exp2_poly2(p0, p1, x0, x1);
-                                ptx::exp2_poly2(p2, p3, x2, x3);
-                            } else {
-                                p0 = ptx::ex2(x0);
-                                p1 = ptx::ex2(x1);
-                                p2 = ptx::ex2(x2);
-                                p3 = ptx::ex2(x3);
-                            }
+                            const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+                            const float p2 = ptx::ex2(x2), p3 = ptx::ex2(x3);
                             wd[k] = pack_e4m3x4(p0, p1, p2, p3);
                             ptx::add2(a0, a1, a0, a1, p0, p1);
                             ptx::add2(a0, a1, a0, a1, p2, p3);

@@ -68,26 +68,6 @@ constexpr float kStaleMaxBound = 1048576.0f;  // 2^20: largest p accepted agains
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz
 constexpr int kSchedDepth = 2;              // unit ring between the producer and the other roles
 constexpr int kHeadGroup = 8;               // heads whose units are interleaved in the queue
-// Softmax tuning knobs (compile-time; -D overrides for experiments).
-#ifndef FA_POLY_PAIRS_PER8
-#define FA_POLY_PAIRS_PER8 0  // measured slower on this kernel than all-MUFU; kept as a tuning knob
-#endif
-#ifndef FA_ROWSUM_BF16
-#define FA_ROWSUM_BF16 1
-#endif
-#ifndef FA_KV_SLOTS_D128
-#define FA_KV_SLOTS_D128 4
-#endif
-#ifndef FA_PACKED_F32X2
-#define FA_PACKED_F32X2 1
-#endif
-#ifndef FA_EARLY_K
-#define FA_EARLY_K 1
-#endif
-constexpr bool kEarlyK = FA_EARLY_K != 0;             // acquire K_{j+1} before waiting for P_0(j)
-constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;  // of every 8 column pairs, this many use exp2_poly2
-constexpr bool kRowsumBf16 = FA_ROWSUM_BF16 != 0;   // normalise O by the sum of the bf16-rounded P
-constexpr bool kPackedF32x2 = FA_PACKED_F32X2 != 0; // packed two-lane fp32 FMA/ADD
 
 template <int D>
 struct Layout {
@@ -95,7 +75,7 @@ struct Layout {
     static constexpr int kHalves = D / 64;                     // 64-column (128-byte) swizzle panels
     static constexpr int kPanelBytes = kBlockM * 128;          // one panel of a 128-row tile
     static constexpr int kTileBytes = kPanelBytes * kHalves;   // a whole 128 x D bf16 tile
-    static constexpr int kSlots = (D == 128) ? FA_KV_SLOTS_D128 : 8;  // K/V ring slots
+    static constexpr int kSlots = (D == 128) ? 4 : 8;          // K/V ring slots
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = kQOff + kTilesPerUnit * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
@@ -448,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_all(kv_full(sv), pv);
                 if (!ok) break;
                 const bool more = j + 1 < n1;
-                if (more && kEarlyK) {
+                if (more) {
                     next_slot(sk, pk);
                     ok = wait_all(kv_full(sk), pk);
                     if (!ok) break;
@@ -460,12 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_after_sync();
                     issue_pv(0, sv, j > 0);
                     if (j == n0 - 1) commit(o_full(0));
-                }
-                if (more && !kEarlyK) {
-                    next_slot(sk, pk);
-                    ok = wait_all(kv_full(sk), pk);
-                    if (!ok) break;
-                    ptx::tc_fence_after_sync();
                 }
                 if (j + 1 < n0) {
                     issue_s(0, sk);
@@ -584,16 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int r = 0; r < 2; ++r) {
                             float x0, x1, p0, p1;
                             ptx::fma2(x0, x1, s[4 * k + 2 * r], s[4 * k + 2 * r + 1], slv, slv, neg_m[r], neg_m[r]);
-                            if (!need_mask && ((2 * k + r) & 7) < kPolyPairsPer8) {
-                                ptx::exp2_poly2(p0, p1, x0, x1);
-                            } else {
-                                p0 = ptx::ex2(x0);
-                                p1 = ptx::ex2(x1);
-                            }
+                            p0 = ptx::ex2(x0);
+                            p1 = ptx::ex2(x1);
                             const uint32_t v = ptx::pack_bf16x2(p0, p1);
                             pk[2 * k + r] = v;
                             ptx::add2(a[r][0], a[r][1], a[r][0], a[r][1], p0, p1);
-                            if (kRowsumBf16) ptx::add_bf16x2_to_f32(b[r][0], b[r][1], v);
+                            ptx::add_bf16x2_to_f32(b[r][0], b[r][1], v);
                         }
                     }
                 };
@@ -640,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     l_run[r] = l_run[r] * alpha[r] + (a[r][0] + a[r][1]);
-                    lb_run[r] = lb_run[r] * alpha[r] + (kRowsumBf16 ? (b[r][0] + b[r][1]) : (a[r][0] + a[r][1]));
+                    lb_run[r] = lb_run[r] * alpha[r] + (b[r][0] + b[r][1]);
                 }
                 ptx::tmem_st16x128b_x16(tmem_s, pk);
 
