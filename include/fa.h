@@ -250,10 +250,16 @@ size_t fa_decode_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t Nk, i
  *                     wrote them); lse device [B][H][N] fp32.
  *   dq, dk, dv        device, [B][H][N][d] bf16, written once.
  *   workspace         device scratch of fa_bwd_workspace_bytes(B, H, N, d)
- *                     bytes (D for every row), 16-byte aligned.
+ *                     bytes, 16-byte aligned: per row (padded to whole
+ *                     128-row blocks) D and -lse*log2(e), and an fp32
+ *                     accumulator for dq ([B*H][N rounded up to 128][d]);
+ *                     its contents on entry do not matter.
  *   scale, causal     as for fa_fwd; dtype must be FA_DTYPE_BF16
  *                     (FA_ERR_UNSUPPORTED otherwise); d is 64 or 128.
- * No score matrix reaches memory: P is recomputed tile by tile from lse.
+ * No score matrix reaches memory: P is recomputed tile by tile from lse, and
+ * each of the five products runs once per tile pair.  dq is accumulated over
+ * key blocks by fp32 reduce-adds whose order varies from run to run, so dq
+ * is reproducible to fp32 rounding, not bit for bit (dk, dv are).
  * Asynchronous on `stream` (three kernel launches); argument errors are
  * reported before any CUDA call.  Alignment 16 bytes (lse 4).  Outputs and
  * workspace must not overlap the inputs or each other.
@@ -263,7 +269,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int64_t B, int64_t H, int64_t N, int64_t d, float scale, int causal, int dtype,
            void* workspace, size_t workspace_bytes, void* stream);
 
-/* fa_bwd_workspace_bytes -- the workspace fa_bwd needs (0 for invalid sizes). */
+/* fa_bwd_workspace_bytes -- the workspace fa_bwd needs (0 for invalid sizes,
+ * including d other than 64 or 128). */
 size_t fa_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
 /*

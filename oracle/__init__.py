@@ -73,6 +73,11 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     b.restype = ctypes.c_int
     b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    br = lib.oracle_attention_bwd_rows
+    br.restype = ctypes.c_int
+    br.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     m = lib.oracle_lse_merge
     m.restype = ctypes.c_int
     m.argtypes = [ctypes.c_void_p] * 2 + [ctypes.c_int64] * 3 + [ctypes.c_void_p] * 2
@@ -167,6 +172,34 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool, lib=None):
                                   float(scale), int(bool(causal)), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
     if rc != 0:
         raise RuntimeError(f"oracle_attention_bwd failed with code {rc}")
+    return dq, dk, dv
+
+
+def attention_bwd_rows(q, k, v, do, scale: float, causal: bool, qrows, krows, lib=None):
+    """The gradients of attention_bwd for chosen rows only, in fp64, for heads
+    too long for the n x n matrices.
+
+    q, k, v, do: [B, H, N, d] (exact input values, fp32).  qrows [B, H, nq]
+    and krows [B, H, nk]: int row indices per head.  Returns (dq [B, H, nq, d]
+    for the query rows, dk, dv [B, H, nk, d] for the key rows), fp64.
+    """
+    lib = lib or load()
+    q, k, v, do = (np.ascontiguousarray(x, dtype=np.float32) for x in (q, k, v, do))
+    if q.ndim != 4 or not (q.shape == k.shape == v.shape == do.shape):
+        raise ValueError("q, k, v, do must share one [B, H, N, d] shape")
+    B, H, N, d = q.shape
+    qrows = np.ascontiguousarray(qrows, dtype=np.int64)
+    krows = np.ascontiguousarray(krows, dtype=np.int64)
+    if qrows.ndim != 3 or qrows.shape[:2] != (B, H) or krows.ndim != 3 or krows.shape[:2] != (B, H):
+        raise ValueError("qrows and krows must be [B, H, count]")
+    nq, nk = qrows.shape[2], krows.shape[2]
+    dq = np.empty((B, H, nq, d), dtype=np.float64)
+    dk, dv = (np.empty((B, H, nk, d), dtype=np.float64) for _ in range(2))
+    rc = lib.oracle_attention_bwd_rows(q.ctypes.data, k.ctypes.data, v.ctypes.data, do.ctypes.data, B * H, N, d,
+                                       float(scale), int(bool(causal)), qrows.ctypes.data, nq, krows.ctypes.data,
+                                       nk, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_bwd_rows failed with code {rc}")
     return dq, dk, dv
 
 

@@ -326,6 +326,135 @@ int oracle_attention_bwd(const float* q, const float* k, const float* v, const f
 }
 
 /*
+ * oracle_attention_bwd_rows -- the gradients of oracle_attention_bwd for
+ * chosen rows only: dq for query rows qrows[h][0..nq) and dk, dv for key rows
+ * krows[h][0..nk) of each head, for heads too long for the n x n matrices
+ * (three fp64 8192 x 8192 matrices take 1.6 GB).  The same definition,
+ * written element by element:
+ *
+ *     s_ij  = scale * q_i . k_j             (j <= i under the causal mask)
+ *     lse_i = m_i + log sum_j exp(s_ij - m_i),  m_i = max_j s_ij   (two passes)
+ *     P_ij  = exp(s_ij - lse_i),   O_i = sum_j P_ij v_j,   D_i = dO_i . O_i
+ *     dP_ij = dO_i . v_j,          dS_ij = P_ij (dP_ij - D_i)
+ *     dq_i  = scale sum_j dS_ij k_j
+ *     dv_j  = sum_i P_ij dO_i,     dk_j  = scale sum_i dS_ij q_i
+ *
+ * Every key's gradients sum over all the queries that see it, so lse and D
+ * come first for every row of the head (one pass over all scores); each
+ * chosen row then costs O(n d).
+ *   q, k, v, dout: [bh][n][d] fp32;  qrows [bh][nq], krows [bh][nk] int64
+ *   dq [bh][nq][d], dk, dv [bh][nk][d] fp64
+ * Returns 0 on success, -1 on bad arguments, -2 if scratch cannot be allocated.
+ */
+int oracle_attention_bwd_rows(const float* q, const float* k, const float* v, const float* dout,
+                              int64_t bh, int64_t n, int64_t d, double scale, int causal,
+                              const int64_t* qrows, int64_t nq, const int64_t* krows, int64_t nk,
+                              double* dq, double* dk, double* dv) {
+    if (!q || !k || !v || !dout || (nq > 0 && (!qrows || !dq)) || (nk > 0 && (!krows || !dk || !dv))) return -1;
+    if (bh <= 0 || n <= 0 || d <= 0 || nq < 0 || nk < 0) return -1;
+    for (int64_t i = 0; i < bh * nq; ++i)
+        if (qrows[i] < 0 || qrows[i] >= n) return -1;
+    for (int64_t i = 0; i < bh * nk; ++i)
+        if (krows[i] < 0 || krows[i] >= n) return -1;
+    double* lse = (double*)malloc((size_t)n * sizeof(double));
+    double* dsum = (double*)malloc((size_t)n * sizeof(double));
+    if (!lse || !dsum) {
+        free(lse);
+        free(dsum);
+        return -2;
+    }
+    int failed = 0;
+    for (int64_t h = 0; h < bh && !failed; ++h) {
+        const float* qh = q + h * n * d;
+        const float* kh = k + h * n * d;
+        const float* vh = v + h * n * d;
+        const float* gh = dout + h * n * d;
+#pragma omp parallel
+        {
+            double* srow = (double*)malloc((size_t)n * sizeof(double));
+            double* orow = (double*)malloc((size_t)d * sizeof(double));
+            if (!srow || !orow) {
+#pragma omp atomic write
+                failed = 1;
+            }
+#pragma omp barrier
+            if (!failed) {
+                /* lse_i and D_i for every query row */
+#pragma omp for schedule(dynamic, 16)
+                for (int64_t i = 0; i < n; ++i) {
+                    const int64_t jend = causal ? i + 1 : n;
+                    double m = -INFINITY;
+                    for (int64_t j = 0; j < jend; ++j) {
+                        double acc = 0.0;
+                        for (int64_t t = 0; t < d; ++t) acc += (double)qh[i * d + t] * (double)kh[j * d + t];
+                        srow[j] = scale * acc;
+                        m = srow[j] > m ? srow[j] : m;
+                    }
+                    double l = 0.0;
+                    for (int64_t j = 0; j < jend; ++j) l += exp(srow[j] - m);
+                    lse[i] = m + log(l);
+                    for (int64_t t = 0; t < d; ++t) orow[t] = 0.0;
+                    for (int64_t j = 0; j < jend; ++j) {
+                        const double pij = exp(srow[j] - lse[i]);
+                        for (int64_t t = 0; t < d; ++t) orow[t] += pij * (double)vh[j * d + t];
+                    }
+                    double acc = 0.0;
+                    for (int64_t t = 0; t < d; ++t) acc += (double)gh[i * d + t] * orow[t];
+                    dsum[i] = acc;
+                }
+                /* dq for the chosen query rows */
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t r = 0; r < nq; ++r) {
+                    const int64_t i = qrows[h * nq + r];
+                    const int64_t jend = causal ? i + 1 : n;
+                    double* out = dq + (h * nq + r) * d;
+                    for (int64_t t = 0; t < d; ++t) out[t] = 0.0;
+                    for (int64_t j = 0; j < jend; ++j) {
+                        double s = 0.0, dp = 0.0;
+                        for (int64_t t = 0; t < d; ++t) {
+                            s += (double)qh[i * d + t] * (double)kh[j * d + t];
+                            dp += (double)gh[i * d + t] * (double)vh[j * d + t];
+                        }
+                        const double pij = exp(scale * s - lse[i]);
+                        const double dsij = pij * (dp - dsum[i]);
+                        for (int64_t t = 0; t < d; ++t) out[t] += dsij * (double)kh[j * d + t];
+                    }
+                    for (int64_t t = 0; t < d; ++t) out[t] *= scale;
+                }
+                /* dk, dv for the chosen key rows */
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t r = 0; r < nk; ++r) {
+                    const int64_t j = krows[h * nk + r];
+                    const int64_t ibeg = causal ? j : 0;
+                    double* okv = dv + (h * nk + r) * d;
+                    double* okk = dk + (h * nk + r) * d;
+                    for (int64_t t = 0; t < d; ++t) okv[t] = okk[t] = 0.0;
+                    for (int64_t i = ibeg; i < n; ++i) {
+                        double s = 0.0, dp = 0.0;
+                        for (int64_t t = 0; t < d; ++t) {
+                            s += (double)qh[i * d + t] * (double)kh[j * d + t];
+                            dp += (double)gh[i * d + t] * (double)vh[j * d + t];
+                        }
+                        const double pij = exp(scale * s - lse[i]);
+                        const double dsij = pij * (dp - dsum[i]);
+                        for (int64_t t = 0; t < d; ++t) {
+                            okv[t] += pij * (double)gh[i * d + t];
+                            okk[t] += dsij * (double)qh[i * d + t];
+                        }
+                    }
+                    for (int64_t t = 0; t < d; ++t) okk[t] *= scale;
+                }
+            }
+            free(srow);
+            free(orow);
+        }
+    }
+    free(lse);
+    free(dsum);
+    return failed ? -2 : 0;
+}
+
+/*
  * oracle_lse_merge -- combine attention results computed over disjoint key
  * sets into the result over their union.  Each part i gives, per query row,
  * o_i = sum_j exp(s_j - lse_i) v_j / 1 over its keys and lse_i = ln sum_j

@@ -437,6 +437,45 @@ def pin_bwd_invariants(lib):
             np.testing.assert_allclose(c, 2 * a - 3 * b, atol=1e-11)
 
 
+def _bwd_rows(lib, q, k, v, do, scale, causal, qrows, krows):
+    return oracle.attention_bwd_rows(q, k, v, do, scale, causal, qrows, krows, lib=lib)
+
+
+def pin_bwd_rows_torch_autograd(lib):
+    """The row-sampled gradients against torch's fp64 autograd through its
+    math attention, on rows that include the first and last of each head; the
+    last case spreads the scores over about +-1000, where exp without the row
+    max overflows."""
+    for (B, H, N, d, causal, seed, scale) in [(1, 2, 41, 8, False, 120, 0.45), (2, 1, 67, 16, True, 121, 0.45),
+                                              (1, 1, 30, 8, True, 122, 40.0)]:
+        q, k, v, do = (_rand((B, H, N, d), seed + i) for i in range(4))
+        g = np.random.default_rng(seed)
+        qrows = np.stack([np.stack([np.r_[0, N - 1, g.choice(N, 5, replace=False)] for _ in range(H)])
+                          for _ in range(B)])
+        krows = np.stack([np.stack([np.r_[N - 1, 0, g.choice(N, 4, replace=False)] for _ in range(H)])
+                          for _ in range(B)])
+        dq, dk, dv = _bwd_rows(lib, q, k, v, do, scale, causal, qrows, krows)
+        tq, tk, tv = (torch.from_numpy(x.astype(np.float64)).requires_grad_() for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+        o.backward(torch.from_numpy(do.astype(np.float64)))
+        for got, full, rows in ((dq, tq.grad, qrows), (dk, tk.grad, krows), (dv, tv.grad, krows)):
+            want = np.take_along_axis(full.numpy(), rows[..., None], axis=2)
+            np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def pin_bwd_rows_match_full_gradients(lib):
+    """The row-sampled gradients equal the full-matrix oracle's rows, on a
+    head with a ragged length and on every row of a small one."""
+    for (N, causal, seed) in [(37, True, 130), (37, False, 131), (12, True, 132)]:
+        q, k, v, do = (_rand((1, 2, N, 8), seed + i) for i in range(4))
+        rows = np.broadcast_to(np.arange(N), (1, 2, N)).copy()
+        dq, dk, dv = _bwd(lib, q, k, v, do, 0.6, causal)
+        rq, rk, rv = _bwd_rows(lib, q, k, v, do, 0.6, causal, rows, rows[:, :, ::-1].copy())
+        np.testing.assert_allclose(rq, dq, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(rk, dk[:, :, ::-1], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(rv, dv[:, :, ::-1], rtol=0, atol=1e-12)
+
+
 # ------------------------------------------------- merging partial results
 def pin_merge_is_attention_over_the_union(lib):
     """Attention over a key set split into parts, merged by log-sum-exp,
@@ -468,7 +507,8 @@ def pin_merge_is_attention_over_the_union(lib):
     np.testing.assert_allclose(lse3, parts_l[0], rtol=0, atol=1e-6)
 
 
-BWD_PINS = [pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants]
+BWD_PINS = [pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants, pin_bwd_rows_torch_autograd,
+            pin_bwd_rows_match_full_gradients]
 
 DECODE_PINS = [pin_decode_hand_worked, pin_decode_closed_forms, pin_decode_is_the_last_rows_of_prefill,
                pin_decode_future_keys_ignored, pin_decode_torch_sdpa]

@@ -53,6 +53,17 @@ MUTANTS = [
      "const double w = exp((double)lse_parts[i * rows + r]);"),
     ("merge_lse_without_max", "lse[r] = big + log(tot);", "lse[r] = log(tot);"),
     ("merge_not_normalised", "for (int64_t t = 0; t < d; ++t) o[r * d + t] /= tot;", ""),
+    # the row-sampled backward
+    ("bwd_rows_dq_scale_dropped", "for (int64_t t = 0; t < d; ++t) out[t] *= scale;", ""),
+    ("bwd_rows_dk_scale_dropped", "for (int64_t t = 0; t < d; ++t) okk[t] *= scale;", ""),
+    ("bwd_rows_max_from_first_key_only", "m = srow[j] > m ? srow[j] : m;", "m = j == 0 ? srow[j] : m;"),
+    ("bwd_rows_lse_without_max", "lse[i] = m + log(l);", "lse[i] = log(l);"),
+    ("bwd_rows_no_softmax_jacobian", "const double dsij = pij * (dp - dsum[i]);\n                        for (int64_t t = 0; t < d; ++t) out[t]",
+     "const double dsij = pij * dp;\n                        for (int64_t t = 0; t < d; ++t) out[t]"),
+    ("bwd_rows_key_mask_off", "const int64_t ibeg = causal ? j : 0;", "const int64_t ibeg = 0;"),
+    ("bwd_rows_key_diagonal_dropped", "const int64_t ibeg = causal ? j : 0;", "const int64_t ibeg = causal ? j + 1 : 0;"),
+    ("bwd_rows_dv_with_q", "okv[t] += pij * (double)gh[i * d + t];", "okv[t] += pij * (double)qh[i * d + t];"),
+    ("bwd_rows_d_from_v", "acc += (double)gh[i * d + t] * orow[t];", "acc += (double)gh[i * d + t] * (double)vh[i * d + t];"),
     ("bwd_dp_with_k", "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)vh[c * d + t];",
      "for (int64_t t = 0; t < d; ++t) acc += (double)gh[r * d + t] * (double)kh[c * d + t];"),
 ]

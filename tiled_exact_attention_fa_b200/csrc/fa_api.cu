@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cmath>
@@ -786,59 +787,98 @@ extern "C" int fa_decode(const void* q, const void* k, const void* v, void* o, f
 }
 
 // ---------------------------------------------------------------------------
-// fa_bwd: gradients (see fa_bwd_tc.cuh).  Workspace: D = rowsum(dO * O),
-// [B*H][N] fp32.
+// fa_bwd: gradients (see fa_bwd_tc.cuh).  Workspace, every array padded to
+// whole 128-row blocks per head (npad rows): L = -lse * log2(e) and
+// D = rowsum(dO * O), [B*H][npad] fp32 each, then the fp32 dQ accumulator
+// [B*H][npad][d].
 namespace {
+
+struct BwdWorkspace {
+    size_t vec_bytes = 0;  // one of the two row vectors, rounded up to 256
+    size_t total = 0;
+};
+
+BwdWorkspace bwd_workspace_layout(int64_t bh, int64_t npad, int64_t d) {
+    BwdWorkspace w;
+    w.vec_bytes = round_up(static_cast<size_t>(bh * npad) * 4, 256);
+    w.total = 2 * w.vec_bytes + round_up(static_cast<size_t>(bh * npad * d) * 4, 256);
+    return w;
+}
+
+// 3-D view (d, npad, B*H) of the fp32 dQ accumulator, boxes of 32 columns x
+// 32 rows with 128-byte swizzle: the unit of the kernel's reduce-adds.
+int encode_dq_acc_map(CUtensorMap* map, float* ptr, int64_t bh, int64_t npad, int64_t d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(npad), static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 4), static_cast<cuuint64_t>(npad * d * 4)};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (dQ accumulator) failed with CUresult " + std::to_string(r));
+    return FA_OK;
+}
 
 template <int D, bool kCausal>
 int launch_bwd(DeviceState* st, int slot, const void* q, const void* k, const void* v, const void* o,
-               const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dsum, int64_t bh,
+               const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace, int64_t bh,
                int64_t n, float scale, cudaStream_t s) {
     using L = fa::bwd::Layout<D>;
-    auto kdq = fa::bwd::fa_bwd_dq_kernel<D, kCausal>;
-    auto kkv = fa::bwd::fa_bwd_dkdv_kernel<D, kCausal>;
+    auto kernel = fa::bwd::fa_bwd_kernel<D, kCausal>;
     cudaError_t e;
     if (!st->bwd_smem_raised[slot]) {
-        if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes)) != cudaSuccess)
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes)) != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
         std::lock_guard<std::mutex> lock(g_mu);
         st->bwd_smem_raised[slot] = true;
     }
-    const int64_t rows = bh * n;
-    fa::bwd::fa_bwd_dot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), dsum, rows);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the backward row-dot kernel");
-    CUtensorMap tq, tk, tv, tdo;
+    const int64_t nblocks = (n + fa::bwd::kBlock - 1) / fa::bwd::kBlock;
+    const int64_t npad = nblocks * fa::bwd::kBlock;
+    const BwdWorkspace ws = bwd_workspace_layout(bh, npad, D);
+    float* lvec = static_cast<float*>(workspace);
+    float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.vec_bytes);
+    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ws.vec_bytes);
+    const int64_t prows = bh * npad;
+    fa::bwd::fa_bwd_prep_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), lse, lvec, dvec, dq_acc, bh,
+        static_cast<int>(n), static_cast<int>(npad));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the backward preparation kernel");
+    CUtensorMap tq, tk, tv, tdo, tdq;
     int rc;
     if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK || (rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK ||
-        (rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK || (rc = encode_tile_map(&tdo, dout, bh, n, D)) != FA_OK)
+        (rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK || (rc = encode_tile_map(&tdo, dout, bh, n, D)) != FA_OK ||
+        (rc = encode_dq_acc_map(&tdq, dq_acc, bh, npad, D)) != FA_OK)
         return rc;
     fa::bwd::Params p;
-    p.lse = lse;
-    p.dsum = dsum;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.lvec = lvec;
+    p.dvec = dvec;
     p.status = st->status;
     p.n = static_cast<int>(n);
-    p.nblocks = static_cast<int>((n + fa::bwd::kBlock - 1) / fa::bwd::kBlock);
+    p.npad = static_cast<int>(npad);
+    p.nblocks = static_cast<int>(nblocks);
+    p.bh = static_cast<int>(bh);
     p.scale = scale;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    dim3 grid(static_cast<unsigned>(p.nblocks), static_cast<unsigned>(bh));
-    p.out0 = static_cast<__nv_bfloat16*>(dq);
-    p.out1 = nullptr;
-    kdq<<<grid, fa::bwd::kThreads, L::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the dQ kernel");
-    p.out0 = static_cast<__nv_bfloat16*>(dv);
-    p.out1 = static_cast<__nv_bfloat16*>(dk);
-    kkv<<<grid, fa::bwd::kThreads, L::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the dK/dV kernel");
+    kernel<<<static_cast<unsigned>(nblocks * bh), fa::bwd::kThreads, L::kSmemBytes, s>>>(tq, tk, tv, tdo, tdq, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the backward kernel");
+    const int64_t vecs = bh * n * (D / 8);
+    const int64_t cap = static_cast<int64_t>(st->sm_count) * 8;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((vecs + 255) / 256, cap));
+    fa::bwd::fa_bwd_dq_convert_kernel<D><<<blocks, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), bh,
+                                                                static_cast<int>(n), static_cast<int>(npad), scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the dQ conversion kernel");
     return FA_OK;
 }
 
 }  // namespace
 
 extern "C" size_t fa_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
-    if (B < 1 || H < 1 || N < 1 || d < 1 || B > (int64_t{1} << 24) / H || N > (int64_t{1} << 30)) return 0;
-    return round_up(static_cast<size_t>(B * H * N) * 4, 256);
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128) || B > (int64_t{1} << 24) / H || N > (int64_t{1} << 30))
+        return 0;
+    const int64_t npad = (N + fa::bwd::kBlock - 1) / fa::bwd::kBlock * fa::bwd::kBlock;
+    return bwd_workspace_layout(B * H, npad, d).total;
 }
 
 extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -853,6 +893,8 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
     if (dtype != FA_DTYPE_BF16) return fail(FA_ERR_UNSUPPORTED, "the backward pass takes bf16 tensors");
     if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
     if (N > (int64_t{1} << 30) || B > 65535 / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H or N too large");
+    if ((N + fa::bwd::kBlock - 1) / fa::bwd::kBlock * B * H > INT_MAX)
+        return fail(FA_ERR_INVALID_ARGUMENT, "B * H * N too large");
     const int64_t bh = B * H;
     const size_t tb = static_cast<size_t>(bh * N * d * 2), lb = static_cast<size_t>(bh * N * 4);
     const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
@@ -879,12 +921,11 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
     if (rc != FA_OK) return rc;
     if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the backward kernels need an sm_100 (B200-class) GPU");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float* dsum = static_cast<float*>(workspace);
     const bool c = causal != 0;
-    if (d == 128) return c ? launch_bwd<128, true>(st, 0, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s)
-                           : launch_bwd<128, false>(st, 1, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
-    return c ? launch_bwd<64, true>(st, 2, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s)
-             : launch_bwd<64, false>(st, 3, q, k, v, o, lse, dout, dq, dk, dv, dsum, bh, N, scale, s);
+    if (d == 128) return c ? launch_bwd<128, true>(st, 0, q, k, v, o, lse, dout, dq, dk, dv, workspace, bh, N, scale, s)
+                           : launch_bwd<128, false>(st, 1, q, k, v, o, lse, dout, dq, dk, dv, workspace, bh, N, scale, s);
+    return c ? launch_bwd<64, true>(st, 2, q, k, v, o, lse, dout, dq, dk, dv, workspace, bh, N, scale, s)
+             : launch_bwd<64, false>(st, 3, q, k, v, o, lse, dout, dq, dk, dv, workspace, bh, N, scale, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -12,24 +12,37 @@
 // tensor memory (TMEM) and the softmax statistics come from the saved lse.
 //
 // Three kernels:
-//   * fa_bwd_dot_kernel: D = rowsum(dO * O), one warp per row;
-//   * fa_bwd_dq_kernel: one CTA per (head, 128-row query block) walks the KV
-//     blocks: S = Q K_j^T and dP = dO V_j^T into TMEM, the compute warps turn
-//     them into dS (bf16, into free TMEM columns), then dQ += dS K_j in TMEM;
-//   * fa_bwd_dkdv_kernel: one CTA per (head, 128-key block) walks the query
-//     blocks: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM, the compute warps
-//     write P^T and dS^T (bf16) over them, then dV += P^T dO_i and
-//     dK += dS^T Q_i in TMEM.
-// S and dP are computed in both kernels (so dQ needs no atomics across
-// CTAs); that is 14 instead of 10 units of N^2 d work.  Roles per CTA: warps
-// 0-7 compute (one TMEM lane = one row per thread; the two warps of a lane
-// quarter take one half of the 128 columns each), warp 8 issues
-// tcgen05.mma from one elected lane, warp 9 streams tiles with TMA through a
-// 4-slot shared-memory ring.  All operand forms are the forward's: K-major
-// shared-memory operands (Q, K, V, dO with d contiguous), MN-major B operands
-// for the products over rows (K, Q, dO as [rows][d]), and A from TMEM.
-// Every mbarrier wait is bounded (status word, abort flag, drain), as in the
-// forward.
+//   * fa_bwd_prep_kernel: per row, D = rowsum(dO * O) and L = -lse * log2(e)
+//     (padded to whole 128-row blocks: L = -inf, D = 0 past the end), and the
+//     row of the fp32 dQ accumulator set to zero;
+//   * fa_bwd_kernel: one CTA per (head, 128-key block) walks the query blocks
+//     i it can see.  With K and V resident in shared memory, per block:
+//         S^T  = K Q_i^T          -> TMEM        (M = keys, N = queries)
+//         dP^T = V dO_i^T         -> TMEM
+//         P^T  = 2^(S^T * scale * log2 e + L_i)   (compute warps; bf16 back
+//                                                  into TMEM over S^T)
+//         dS^T = P^T * (dP^T - D_i)               (compute warps; bf16 into
+//                                                  shared memory, once)
+//         dV  += P^T dO_i         (A from TMEM)
+//         dK  += dS^T Q_i         (A = the dS tile, K-major)
+//         dQ_i = dS K             (A = the same tile read MN-major) -> TMEM
+//     and four drain warps move each dQ_i out of TMEM into shared memory and
+//     add it into the fp32 accumulator with TMA bulk reduce-adds, so every
+//     product runs once: 10 units of N^2 d on the tensor core;
+//   * fa_bwd_dq_convert_kernel: dQ = scale * accumulator, to bf16.
+//
+// Roles of fa_bwd_kernel: warps 0-7 compute (one TMEM lane = one key row per
+// thread; the two warps of a lane quarter take one half of the 128 query
+// columns each), warp 8 issues tcgen05.mma from one elected lane, warp 9
+// streams Q_i (with its L and D slices) and dO_i with TMA, warps 10-13 drain
+// dQ.  The MMA warp's order per block i keeps the tensor core fed while the
+// compute warps work:
+//     dV(i), S^T(i+1), dQ(i), dK(i), dP^T(i+1)
+// S^T(i+1) goes over P^T(i) once dV(i) has read it (the tensor core runs one
+// thread's MMAs in issue order); dQ(i) lands in the columns of dP^T(i), which
+// the compute warps have read by then, and dP^T(i+1) follows once the drain
+// warps have read dQ(i) -- while dK(i) runs.  Every mbarrier wait is bounded
+// (status word, abort flag, drain), as in the forward.
 #pragma once
 
 #include <cstdint>
@@ -42,142 +55,116 @@
 namespace fa {
 namespace bwd {
 
-constexpr int kBlock = 128;       // rows (queries or keys) per tile
-constexpr int kComputeWarps = 8;  // two per TMEM lane quarter, one half of the columns each
+constexpr int kBlock = 128;        // rows (queries or keys) per tile
+constexpr int kComputeWarps = 8;   // two per TMEM lane quarter, one half of the query columns each
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
-constexpr int kThreads = 320;
-constexpr int kSlots = 4;         // streamed tiles in flight
+constexpr int kDrainWarp0 = 10;
+constexpr int kDrainWarps = 4;     // one per lane quarter of the dQ tile
+constexpr int kThreads = 32 * (kDrainWarp0 + kDrainWarps);
+constexpr int kQSlots = 2;         // Q_i tiles in flight (each with its L and D slices)
+constexpr int kStageBytes = 32 * 128;  // one drain warp's 32 rows x 32 fp32 columns
 constexpr uint32_t kTmemCols = 512;
+constexpr int kHeadGroup = 8;      // heads whose key blocks are interleaved in the launch order
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Layout {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kHalves = D / 64;
-    static constexpr int kPanelBytes = kBlock * 128;
-    static constexpr int kTileBytes = kPanelBytes * kHalves;
-    static constexpr int kAOff = 0;                                 // resident tile A (Q or K)
-    static constexpr int kBOff = kTileBytes;                        // resident tile B (dO or V)
-    static constexpr int kRingOff = 2 * kTileBytes;
-    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    // a_full, b_full, full[S], empty[S], s_full, p_full, done, drain, sdp_free, p_full_odd
-    static constexpr int kNumBars = 2 + 2 * kSlots + 6;
+    static constexpr int kPanelBytes = kBlock * 128;            // 128 rows x 64 bf16
+    static constexpr int kTileBytes = kPanelBytes * kHalves;    // 128 x D bf16
+    static constexpr int kDoSlots = D == 64 ? 2 : 1;
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kTileBytes;
+    static constexpr int kQOff = 2 * kTileBytes;
+    static constexpr int kDoOff = kQOff + kQSlots * kTileBytes;
+    static constexpr int kDsOff = kDoOff + kDoSlots * kTileBytes;    // dS^T [key][query] bf16, 2 panels
+    static constexpr int kStageOff = kDsOff + 2 * kPanelBytes;       // drain staging, kStageBytes per warp
+    static constexpr int kVecOff = kStageOff + kDrainWarps * kStageBytes;  // per Q slot: L[128], D[128] fp32
+    static constexpr int kBarOff = kVecOff + kQSlots * 2 * kBlock * 4;
+    // kv_full, q_full[Q], q_empty[Q], do_full[S], do_empty[S],
+    // s_full, dp_full, p_full, ds_full, ds_free, dq_full, dq_free, done, drain
+    static constexpr int kNumBars = 1 + 2 * kQSlots + 2 * kDoSlots + 9;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;         // tmem base, abort flag
-    static constexpr int kVecOff = (kMiscOff + 16 + 15) & ~15;      // float[2][kBlock] (dK/dV kernel)
-    static constexpr int kBytes = kVecOff + 2 * kBlock * 4;
-    static constexpr int kSmemBytes = kBytes + 1024;
-    static constexpr uint32_t kTmemS = 0;        // S or S^T; P^T / dS over its first 64 columns
-    static constexpr uint32_t kTmemDP = 128;     // dP or dP^T; dS^T over its first 64 columns
-    static constexpr uint32_t kTmemAcc0 = 256;   // dQ, or dV
-    static constexpr uint32_t kTmemAcc1 = 256 + D;  // dK
-    static constexpr uint32_t kTmemDS = 384;         // dS of the dQ kernel: two buffers of 64 columns
+    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kSmemBytes = kBytes + 1024;                // slack for 1024-byte alignment
+    static constexpr uint32_t kTmemS = 0;         // S^T fp32; P^T bf16 pairs at [64h, 64h + 32)
+    static constexpr uint32_t kTmemDP = 128;      // dP^T fp32, then dQ_i (M = queries)
+    static constexpr uint32_t kTmemDV = 256;
+    static constexpr uint32_t kTmemDK = 256 + D;
+    static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct Params {
-    __nv_bfloat16* out0;   // dQ (dq kernel) or dV (dkdv kernel)
-    __nv_bfloat16* out1;   // dK (dkdv kernel)
-    const float* lse;      // [bh][n] natural log, from the forward
-    const float* dsum;     // [bh][n] D = rowsum(dO * O)
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    const float* lvec;     // [bh][npad] -lse * log2(e); -inf on padding rows
+    const float* dvec;     // [bh][npad] D = rowsum(dO * O); 0 on padding rows
     int* status;
-    int n;
+    int n;                 // sequence length
+    int npad;              // nblocks * 128
     int nblocks;           // ceil(n / 128)
+    int bh;                // B * H
     float scale;
     float scale_log2;      // scale * log2(e)
 };
 
-// D = rowsum(dO * O) in fp32: one warp per row, lane l takes a d/32 slice.
+// Per row of every head (padded to whole blocks): D, L, and the fp32 dQ
+// accumulator row set to zero.  One warp per row.
 template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* dout, const __nv_bfloat16* o,
-                                                         float* dsum, int64_t rows) {
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const __nv_bfloat16* dout, const __nv_bfloat16* o,
+                                                          const float* lse, float* lvec, float* dvec,
+                                                          float* dq_acc, int64_t bh, int n, int npad) {
+    const int64_t prow = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // padded row index
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
+    if (prow >= bh * npad) return;
+    const int64_t head = prow / npad;
+    const int r = static_cast<int>(prow - head * npad);
     constexpr int kPer = D / 32;
-    const __nv_bfloat16* a = dout + row * D + lane * kPer;
-    const __nv_bfloat16* b = o + row * D + lane * kPer;
     float acc = 0.f;
+    if (r < n) {
+        const int64_t row = head * n + r;
+        const __nv_bfloat16* a = dout + row * D + lane * kPer;
+        const __nv_bfloat16* b = o + row * D + lane * kPer;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) acc = fmaf(__bfloat162float(a[e]), __bfloat162float(b[e]), acc);
+        for (int e = 0; e < kPer; ++e) acc = fmaf(__bfloat162float(a[e]), __bfloat162float(b[e]), acc);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) dsum[row] = acc;
+        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + prow * D);
+#pragma unroll
+    for (int e = lane; e < D / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0) {
+        dvec[prow] = acc;
+        lvec[prow] = r < n ? -lse[head * n + r] * kLog2e : -INFINITY;
+    }
 }
 
-// Shared pieces of the two main kernels.
+// dQ = scale * accumulator, rows < n of each head, to bf16 (8 values per thread).
 template <int D>
-struct Common {
-    using L = Layout<D>;
-    uint32_t base;
-    uint32_t bar0;
-    __device__ uint32_t a_full() const { return bar0; }
-    __device__ uint32_t b_full() const { return bar0 + 8u; }
-    __device__ uint32_t full(int s) const { return bar0 + 8u * (2 + s); }
-    __device__ uint32_t empty(int s) const { return bar0 + 8u * (2 + kSlots + s); }
-    __device__ uint32_t s_full() const { return bar0 + 8u * (2 + 2 * kSlots); }
-    __device__ uint32_t p_full() const { return bar0 + 8u * (3 + 2 * kSlots); }
-    __device__ uint32_t done() const { return bar0 + 8u * (4 + 2 * kSlots); }
-    __device__ uint32_t drain() const { return bar0 + 8u * (5 + 2 * kSlots); }
-    __device__ uint32_t sdp_free() const { return bar0 + 8u * (6 + 2 * kSlots); }
-    // the dQ kernel's dS(j) is signalled on p_full for even j and on this one
-    // for odd j: the compute warps may finish dS(j+1) before the MMA warp has
-    // observed dS(j), and one barrier would then complete two phases unseen
-    __device__ uint32_t p_full_odd() const { return bar0 + 8u * (7 + 2 * kSlots); }
-    __device__ uint32_t p_full_of(int j) const { return (j & 1) ? p_full_odd() : p_full(); }
-    __device__ uint32_t slot_addr(int s) const { return base + L::kRingOff + s * L::kTileBytes; }
-};
-
-// Producer: the two resident tiles of the unit (rows `row0` of maps ra, rb),
-// then, for each streamed block b in [b_begin, b_end), tile b of map sa and
-// tile b of map sb through the ring.  Waits until every copy has landed.
-template <int D>
-__device__ void produce(const Common<D>& c, const fa::tc::Sync& sync, const CUtensorMap* ra,
-                        const CUtensorMap* rb, int row0, const CUtensorMap* sa, const CUtensorMap* sb, int b_begin,
-                        int b_end, int bh) {
-    using L = Layout<D>;
-    const bool leader = ptx::elect_one();
-    const uint64_t keep = ptx::policy_evict_last();
-    if (leader) {
-        ptx::mbar_arrive_expect_tx(c.a_full(), L::kTileBytes);
-        for (int h = 0; h < L::kHalves; ++h)
-            ptx::tma_load_3d(c.base + L::kAOff + h * L::kPanelBytes, ra, c.a_full(), h * 64, row0, bh, keep);
-        ptx::mbar_arrive_expect_tx(c.b_full(), L::kTileBytes);
-        for (int h = 0; h < L::kHalves; ++h)
-            ptx::tma_load_3d(c.base + L::kBOff + h * L::kPanelBytes, rb, c.b_full(), h * 64, row0, bh, keep);
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t bh,
+                                                                int n, int npad, float scale) {
+    const int64_t total = bh * n * (D / 8);
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t row = t / (D / 8);
+        const int c = static_cast<int>(t - row * (D / 8)) * 8;
+        const int64_t head = row / n;
+        const int64_t prow = head * npad + (row - head * n);
+        const float4* src = reinterpret_cast<const float4*>(dq_acc + prow * D + c);
+        const float4 a = src[0], b = src[1];
+        uint4 w;
+        w.x = ptx::pack_bf16x2(a.x * scale, a.y * scale);
+        w.y = ptx::pack_bf16x2(a.z * scale, a.w * scale);
+        w.z = ptx::pack_bf16x2(b.x * scale, b.y * scale);
+        w.w = ptx::pack_bf16x2(b.z * scale, b.w * scale);
+        *reinterpret_cast<uint4*>(dq + row * D + c) = w;
     }
-    int slot = 0;
-    uint32_t phase = 0, nloads = 0;
-    bool ok = true;
-    for (int b = b_begin; b < b_end && ok; ++b) {
-        for (int which = 0; which < 2 && ok; ++which) {
-            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.empty(slot), phase ^ 1));
-            if (!ok) break;
-            if (leader) {
-                ptx::mbar_arrive_expect_tx(c.full(slot), L::kTileBytes);
-                const CUtensorMap* m = which == 0 ? sa : sb;
-                for (int h = 0; h < L::kHalves; ++h)
-                    ptx::tma_load_3d(c.slot_addr(slot) + h * L::kPanelBytes, m, c.full(slot), h * 64, b * kBlock, bh,
-                                     keep);
-            }
-            ++nloads;
-            if (++slot == kSlots) {
-                slot = 0;
-                phase ^= 1;
-            }
-        }
-    }
-    // every issued copy lands before shared memory is released
-    for (uint32_t s = 0; s < static_cast<uint32_t>(kSlots) && s < nloads; ++s) {
-        const uint32_t last = s + kSlots * ((nloads - 1 - s) / kSlots);
-        fa::tc::drain_bar(sync, c.full(s), (last / kSlots) & 1);
-    }
-    fa::tc::drain_bar(sync, c.a_full(), 0);
-    fa::tc::drain_bar(sync, c.b_full(), 0);
-    __syncwarp();
 }
 
-// 8 MMAs of K = 16 over the head dim: D[tmem] = A[128 x D] * B[128 x D]^T,
-// both K-major 128-byte-swizzled shared-memory tiles.
+// D[tmem] = A[128 x D] * B[128 x D]^T over the head dim: both K-major
+// 128-byte-swizzled shared-memory tiles (S^T = K Q^T, dP^T = V dO^T).
 template <int D>
 __device__ __forceinline__ void mma_rows_by_rows(bool leader, uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
     using L = Layout<D>;
@@ -189,136 +176,6 @@ __device__ __forceinline__ void mma_rows_by_rows(bool leader, uint32_t d_tmem, u
         const uint32_t off = ((ks >> 2) * L::kPanelBytes + (ks & 3) * 32) >> 4;
         if (leader) ptx::mma_ss(d_tmem, ad + off, bd + off, idesc, ks > 0);
     }
-}
-
-// 8 MMAs of K = 16 over 128 rows: D[tmem, 128 x D] (+)= A[tmem, 128 x 128 bf16]
-// * B[smem, 128 rows x D, MN-major].
-template <int D>
-__device__ __forceinline__ void mma_tmem_by_tile(bool leader, uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
-                                                 bool accumulate) {
-    using L = Layout<D>;
-    constexpr uint32_t idesc = ptx::make_idesc_bf16(kBlock, D, true);
-    const uint64_t bd = ptx::make_smem_desc(b_smem, L::kPanelBytes, 1024);
-#pragma unroll
-    for (int ks = 0; ks < kBlock / 16; ++ks)
-        if (leader)
-            ptx::mma_ts(d_tmem, a_tmem + ks * 8, bd + ((ks * 16 * 128) >> 4), idesc, (accumulate || ks > 0) ? 1u : 0u);
-}
-
-// The dQ kernel's MMA loop, pipelined: as soon as the compute warps have
-// read S(j) and dP(j) (sdp_free), S(j+1) and dP(j+1) are issued over them,
-// so these products run while dS(j) is computed; dS alternates between two
-// TMEM buffers, and dQ += dS(j) K_j follows once dS(j) is in place.  In-order
-// execution makes the reuse safe: dQ(j) is issued before S(j+2), so when the
-// compute warps see S(j+2) complete, dQ(j) has read dS buffer j & 1.
-template <int D>
-__device__ void mma_loop_dq(const Common<D>& c, const fa::tc::Sync& sync, uint32_t tmem, int nb) {
-    using L = Layout<D>;
-    const bool leader = ptx::elect_one();
-    auto wait_all = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, fa::tc::wait_bar(sync, bar, parity));
-    };
-    auto commit = [&](uint32_t bar) {
-        if (leader) ptx::mma_commit(bar);
-    };
-    int slot = 0;
-    uint32_t phase = 0;
-    // the next (K_j, V_j) pair of ring slots
-    auto take = [&](int& xs, uint32_t& xp, int& ys, uint32_t& yp) {
-        xs = slot;
-        ys = slot + 1;
-        xp = yp = phase;
-        slot = (slot + 2) % kSlots;
-        if (slot < 2) phase ^= 1;
-    };
-    auto issue_sdp = [&](int xs, int ys) {
-        mma_rows_by_rows<D>(leader, tmem + L::kTmemS, c.base + L::kAOff, c.slot_addr(xs));   // S = Q K^T
-        mma_rows_by_rows<D>(leader, tmem + L::kTmemDP, c.base + L::kBOff, c.slot_addr(ys));  // dP = dO V^T
-        commit(c.s_full());
-        commit(c.empty(ys));  // V_j is done once dP is
-    };
-    bool ok = wait_all(c.a_full(), 0) && wait_all(c.b_full(), 0);
-    int xs, ys;
-    uint32_t xp, yp;
-    take(xs, xp, ys, yp);
-    ok = ok && wait_all(c.full(xs), xp) && wait_all(c.full(ys), yp);
-    if (ok) {
-        ptx::tc_fence_after_sync();
-        issue_sdp(xs, ys);
-    }
-    int kslot = xs;
-    for (int j = 0; j < nb && ok; ++j) {
-        ok = wait_all(c.sdp_free(), j & 1);
-        if (!ok) break;
-        int next_k = -1;
-        if (j + 1 < nb) {
-            take(xs, xp, ys, yp);
-            ok = wait_all(c.full(xs), xp) && wait_all(c.full(ys), yp);
-            if (!ok) break;
-            ptx::tc_fence_after_sync();
-            issue_sdp(xs, ys);
-            next_k = xs;
-        }
-        ok = wait_all(c.p_full_of(j), (j >> 1) & 1);
-        if (!ok) break;
-        ptx::tc_fence_after_sync();
-        mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemDS + 64 * (j & 1), c.slot_addr(kslot), j > 0);
-        commit(c.empty(kslot));  // K_j is done once dQ(j) is
-        kslot = next_k;
-    }
-    commit(c.done());
-    commit(c.drain());
-    fa::tc::drain_bar(sync, c.drain(), 0);
-    __syncwarp();
-}
-
-// The MMA warp's loop, shared by both kernels (A, B resident; streamed pairs
-// (X_b, Y_b) in the ring):
-//   T0 = A X_b^T   -> kTmemS          T1 = B Y_b^T   -> kTmemDP
-//   wait for the compute warps' bf16 results over T0 and T1
-//   acc0 += R0 * (dq: X_b | dkdv: Y_b),  acc1 += R1 * X_b (dkdv only)
-// where R0 sits over T0 (dS in the dq kernel, P^T in the dK/dV kernel) and
-// R1 over T1 (dS^T, dK/dV kernel only).
-template <int D, bool kDkdv>
-__device__ void mma_loop(const Common<D>& c, const fa::tc::Sync& sync, uint32_t tmem, int nb) {
-    using L = Layout<D>;
-    const bool leader = ptx::elect_one();
-    auto wait_all = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, fa::tc::wait_bar(sync, bar, parity));
-    };
-    auto commit = [&](uint32_t bar) {
-        if (leader) ptx::mma_commit(bar);
-    };
-    bool ok = wait_all(c.a_full(), 0) && wait_all(c.b_full(), 0);
-    int slot = 0;
-    uint32_t phase = 0;
-    for (int b = 0; b < nb && ok; ++b) {
-        const int xs = slot, ys = (slot + 1) % kSlots;
-        const uint32_t xp = phase, yp = (slot + 1 == kSlots) ? phase ^ 1 : phase;
-        slot = (slot + 2) % kSlots;
-        if (slot < 2) phase ^= 1;
-        ok = wait_all(c.full(xs), xp) && wait_all(c.full(ys), yp);
-        if (!ok) break;
-        ptx::tc_fence_after_sync();
-        mma_rows_by_rows<D>(leader, tmem + L::kTmemS, c.base + L::kAOff, c.slot_addr(xs));
-        mma_rows_by_rows<D>(leader, tmem + L::kTmemDP, c.base + L::kBOff, c.slot_addr(ys));
-        commit(c.s_full());
-        ok = wait_all(c.p_full(), b & 1);
-        if (!ok) break;
-        ptx::tc_fence_after_sync();
-        if (kDkdv) {
-            mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemS, c.slot_addr(ys), b > 0);   // dV += P^T dO
-            mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc1, tmem + L::kTmemDP, c.slot_addr(xs), b > 0);  // dK += dS^T Q
-        } else {
-            mma_tmem_by_tile<D>(leader, tmem + L::kTmemAcc0, tmem + L::kTmemDS, c.slot_addr(xs), b > 0);  // dQ += dS K
-        }
-        commit(c.empty(xs));
-        commit(c.empty(ys));
-    }
-    commit(c.done());
-    commit(c.drain());
-    fa::tc::drain_bar(sync, c.drain(), 0);
-    __syncwarp();
 }
 
 // Epilogue: columns [col_begin, col_begin + D/2) of a TMEM accumulator (times
@@ -343,151 +200,67 @@ __device__ __forceinline__ void store_rows(uint32_t tmem_rows, __nv_bfloat16* ro
     }
 }
 
-// ---------------------------------------------------------------- dQ kernel
-// CTA = (query block qb, head bh); tiles: Q, dO resident; K_j, V_j streamed.
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
-    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const Params p) {
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_dq, const Params p) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = blockIdx.x, bh = blockIdx.y;
-    const Common<D> c{base, base + L::kBarOff};
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-    const fa::tc::Sync sync{abort_flag, p.status};
-    const int nb = kCausal ? min(p.nblocks, qb + 1) : p.nblocks;  // KV blocks this query block uses
 
-    if (threadIdx.x == 0) {
-        ptx::mbar_init(c.a_full(), 1);
-        ptx::mbar_init(c.b_full(), 1);
-        for (int s = 0; s < kSlots; ++s) {
-            ptx::mbar_init(c.full(s), 1);
-            ptx::mbar_init(c.empty(s), 1);
-        }
-        ptx::mbar_init(c.s_full(), 1);
-        ptx::mbar_init(c.p_full(), 32 * kComputeWarps);
-        ptx::mbar_init(c.done(), 1);
-        ptx::mbar_init(c.drain(), 1);
-        ptx::mbar_init(c.sdp_free(), 32 * kComputeWarps);
-        ptx::mbar_init(c.p_full_odd(), 32 * kComputeWarps);
-        *abort_flag = 0;
-        ptx::fence_mbar_init();
-    }
-    if (warp == kMmaWarp) {
-        ptx::tmem_alloc(ptx::smem_addr(tmem_base_ptr), kTmemCols);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = *tmem_base_ptr;
-
-    if (warp == kLoadWarp) {
-        produce<D>(c, sync, &tm_q, &tm_do, qb * kBlock, &tm_k, &tm_v, 0, nb, bh);
-    } else if (warp == kMmaWarp) {
-        mma_loop_dq<D>(c, sync, tmem, nb);
-    } else {
-        // one query row per thread (TMEM lane = row within the block); the
-        // warp's half h of the key columns
-        const int q4 = warp & 3, h = warp >> 2;
-        const int r = q4 * 32 + lane;
-        const int row = qb * kBlock + r;
-        const bool valid = row < p.n;
-        const float lse2 = valid ? p.lse[static_cast<int64_t>(bh) * p.n + row] * kLog2e : 0.f;
-        const float drow = valid ? p.dsum[static_cast<int64_t>(bh) * p.n + row] : 0.f;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
-        bool ok = true;
-        for (int j = 0; j < nb && ok; ++j) {
-            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.s_full(), j & 1));
-            if (!ok) break;
-            ptx::tc_fence_after_sync();
-            const uint32_t ds_buf = L::kTmemDS + 64 * (j & 1);
-#pragma unroll
-            for (int cl = 0; cl < kBlock / 2; cl += 32) {
-                const int c0 = h * (kBlock / 2) + cl;
-                uint32_t sv[32], gv[32];
-                ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemS + c0, sv);
-                ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemDP + c0, gv);
-                if (cl + 32 == kBlock / 2) {
-                    // S(j) and dP(j) are in registers: the next pair may overwrite them
-                    ptx::tc_fence_before_sync();
-                    ptx::mbar_arrive(c.sdp_free());
-                }
-                uint32_t ds[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float d2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int key = j * kBlock + c0 + e + u;
-                        const bool use = valid && key < p.n && (!kCausal || key <= row);
-                        const float pr = use ? ptx::ex2(__uint_as_float(sv[e + u]) * p.scale_log2 - lse2) : 0.f;
-                        d2[u] = pr * (__uint_as_float(gv[e + u]) - drow);
-                    }
-                    ds[e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
-                }
-                ptx::tmem_st16(tmem + lane_addr + ds_buf + c0 / 2, ds);
-            }
-            ptx::tmem_st_wait();
-            ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(c.p_full_of(j));
-        }
-        if (ok) ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.done(), 0));
-        if (ok) {
-            ptx::tc_fence_after_sync();
-            store_rows<D>(tmem + lane_addr + L::kTmemAcc0, p.out0 + (static_cast<int64_t>(bh) * p.n + row) * D, valid,
-                          p.scale, h * (D / 2));
-        }
-    }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    if (warp == kMmaWarp) {
-        __syncwarp();
-        ptx::tmem_dealloc(tmem, kTmemCols);
-    }
-}
-
-// ------------------------------------------------------------- dK, dV kernel
-// CTA = (key block kb, head bh); tiles: K, V resident; Q_i, dO_i streamed.
-template <int D, bool kCausal>
-__global__ void __launch_bounds__(kThreads, 1)
-    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const Params p) {
-    using L = Layout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = ptx::smem_addr(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* smem = smem_raw + (base - raw);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kb = blockIdx.x, bh = blockIdx.y;
-    const Common<D> c{base, base + L::kBarOff};
-    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-    float* lse2_sm = reinterpret_cast<float*>(smem + L::kVecOff);  // this query block's lse * log2(e)
-    float* dsum_sm = lse2_sm + kBlock;                              // and its D
-    const fa::tc::Sync sync{abort_flag, p.status};
-    const int i_begin = kCausal ? kb : 0;                           // query blocks that see this key block
+    // CTA -> (key block kb, head bh): heads in groups of kHeadGroup with
+    // their key blocks interleaved (their Q, dO and dQ rows stay in L2); in
+    // each group key block 0 -- under the mask the one that sees the most
+    // query blocks -- comes first.
+    const int per_group = kHeadGroup * p.nblocks;
+    const int grp = blockIdx.x / per_group;
+    const int rem = blockIdx.x - grp * per_group;
+    const int hg = min(kHeadGroup, p.bh - grp * kHeadGroup);
+    const int kb = rem / hg;
+    const int bh = grp * kHeadGroup + (rem - kb * hg);
+    const int i_begin = kCausal ? kb : 0;  // query blocks that see this key block
     const int nb = p.nblocks - i_begin;
 
+    const uint32_t bar0 = base + L::kBarOff;
+    const uint32_t kv_full = bar0;
+    auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto q_empty = [&](int s) { return bar0 + 8u * (1 + kQSlots + s); };
+    auto do_full = [&](int s) { return bar0 + 8u * (1 + 2 * kQSlots + s); };
+    auto do_empty = [&](int s) { return bar0 + 8u * (1 + 2 * kQSlots + L::kDoSlots + s); };
+    const uint32_t ev0 = bar0 + 8u * (1 + 2 * kQSlots + 2 * L::kDoSlots);
+    const uint32_t s_full = ev0, dp_full = ev0 + 8, p_full = ev0 + 16, ds_full = ev0 + 24, ds_free = ev0 + 32,
+                   dq_full = ev0 + 40, dq_free = ev0 + 48, done = ev0 + 56, drain = ev0 + 64;
+    auto q_addr = [&](int s) { return base + L::kQOff + s * L::kTileBytes; };
+    auto do_addr = [&](int s) { return base + L::kDoOff + s * L::kTileBytes; };
+    auto vec_ptr = [&](int s) { return reinterpret_cast<const float*>(smem + L::kVecOff + s * 2 * kBlock * 4); };
+
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+    const fa::tc::Sync sync{abort_flag, p.status};
+
     if (threadIdx.x == 0) {
-        ptx::mbar_init(c.a_full(), 1);
-        ptx::mbar_init(c.b_full(), 1);
-        for (int s = 0; s < kSlots; ++s) {
-            ptx::mbar_init(c.full(s), 1);
-            ptx::mbar_init(c.empty(s), 1);
+        ptx::mbar_init(kv_full, 1);
+        for (int s = 0; s < kQSlots; ++s) {
+            ptx::mbar_init(q_full(s), 1);
+            ptx::mbar_init(q_empty(s), 1);
         }
-        ptx::mbar_init(c.s_full(), 1);
-        ptx::mbar_init(c.p_full(), 32 * kComputeWarps);
-        ptx::mbar_init(c.done(), 1);
-        ptx::mbar_init(c.drain(), 1);
+        for (int s = 0; s < L::kDoSlots; ++s) {
+            ptx::mbar_init(do_full(s), 1);
+            ptx::mbar_init(do_empty(s), 1);
+        }
+        ptx::mbar_init(s_full, 1);
+        ptx::mbar_init(dp_full, 1);
+        ptx::mbar_init(p_full, 32 * kComputeWarps);
+        ptx::mbar_init(ds_full, 32 * kComputeWarps);
+        ptx::mbar_init(ds_free, 1);
+        ptx::mbar_init(dq_full, 1);
+        ptx::mbar_init(dq_free, 32 * kDrainWarps);
+        ptx::mbar_init(done, 1);
+        ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -495,81 +268,312 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_alloc(ptx::smem_addr(tmem_base_ptr), kTmemCols);
         ptx::tmem_relinquish();
     }
+    if (warp == kLoadWarp && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
+        ptx::prefetch_tmap(&tm_do);
+    }
+    if (warp == kDrainWarp0 && lane == 0) ptx::prefetch_tmap(&tm_dq);
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_base_ptr;
 
     if (warp == kLoadWarp) {
-        produce<D>(c, sync, &tm_k, &tm_v, kb * kBlock, &tm_q, &tm_do, i_begin, p.nblocks, bh);
-    } else if (warp == kMmaWarp) {
-        mma_loop<D, true>(c, sync, tmem, nb);
-    } else {
-        // one key row per thread (TMEM lane = key within the block); the
-        // warp's half h of the query columns
-        const int q4 = warp & 3, h = warp >> 2;
-        const int r = q4 * 32 + lane;
-        const int key = kb * kBlock + r;
-        const bool kvalid = key < p.n;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+        // ------------------------------------------------------------ producer
+        const bool leader = ptx::elect_one();
+        const uint64_t keep = ptx::policy_evict_last();  // re-read by the head's other key blocks
+        if (leader) {
+            ptx::mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+            for (int h = 0; h < L::kHalves; ++h) {
+                ptx::tma_load_3d(base + L::kKOff + h * L::kPanelBytes, &tm_k, kv_full, h * 64, kb * kBlock, bh, keep);
+                ptx::tma_load_3d(base + L::kVOff + h * L::kPanelBytes, &tm_v, kv_full, h * 64, kb * kBlock, bh, keep);
+            }
+        }
+        uint32_t nq = 0, ndo = 0;
         bool ok = true;
         for (int b = 0; b < nb && ok; ++b) {
             const int i = i_begin + b;
-            // this query block's statistics, shared by the compute threads
-            asm volatile("bar.sync 1, %0;" ::"r"(32 * kComputeWarps) : "memory");
-            if (h == 0) {
-                const int qrow = i * kBlock + r;
-                const bool qv = qrow < p.n;
-                lse2_sm[r] = qv ? p.lse[static_cast<int64_t>(bh) * p.n + qrow] * kLog2e : 0.f;
-                dsum_sm[r] = qv ? p.dsum[static_cast<int64_t>(bh) * p.n + qrow] : 0.f;
+            const int qs = b % kQSlots;
+            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, q_empty(qs), ((b / kQSlots) & 1) ^ 1));
+            if (!ok) break;
+            if (leader) {
+                ptx::mbar_arrive_expect_tx(q_full(qs), L::kTileBytes + 2 * kBlock * 4);
+                for (int h = 0; h < L::kHalves; ++h)
+                    ptx::tma_load_3d(q_addr(qs) + h * L::kPanelBytes, &tm_q, q_full(qs), h * 64, i * kBlock, bh, keep);
+                const int64_t v0 = static_cast<int64_t>(bh) * p.npad + static_cast<int64_t>(i) * kBlock;
+                const uint32_t vdst = base + L::kVecOff + qs * 2 * kBlock * 4;
+                ptx::bulk_load(vdst, p.lvec + v0, kBlock * 4, q_full(qs), keep);
+                ptx::bulk_load(vdst + kBlock * 4, p.dvec + v0, kBlock * 4, q_full(qs), keep);
             }
-            asm volatile("bar.sync 1, %0;" ::"r"(32 * kComputeWarps) : "memory");
-            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.s_full(), b & 1));
+            ++nq;
+            const int ds = b % L::kDoSlots;
+            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, do_empty(ds), ((b / L::kDoSlots) & 1) ^ 1));
+            if (!ok) break;
+            if (leader) {
+                ptx::mbar_arrive_expect_tx(do_full(ds), L::kTileBytes);
+                for (int h = 0; h < L::kHalves; ++h)
+                    ptx::tma_load_3d(do_addr(ds) + h * L::kPanelBytes, &tm_do, do_full(ds), h * 64, i * kBlock, bh,
+                                     keep);
+            }
+            ++ndo;
+        }
+        // every issued copy lands before shared memory is released
+        for (uint32_t s = 0; s < static_cast<uint32_t>(kQSlots) && s < nq; ++s) {
+            const uint32_t last = s + kQSlots * ((nq - 1 - s) / kQSlots);
+            fa::tc::drain_bar(sync, q_full(s), (last / kQSlots) & 1);
+        }
+        for (uint32_t s = 0; s < static_cast<uint32_t>(L::kDoSlots) && s < ndo; ++s) {
+            const uint32_t last = s + L::kDoSlots * ((ndo - 1 - s) / L::kDoSlots);
+            fa::tc::drain_bar(sync, do_full(s), (last / L::kDoSlots) & 1);
+        }
+        fa::tc::drain_bar(sync, kv_full, 0);
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        const bool leader = ptx::elect_one();
+        auto wait_all = [&](uint32_t bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, fa::tc::wait_bar(sync, bar, parity));
+        };
+        auto commit = [&](uint32_t bar) {
+            if (leader) ptx::mma_commit(bar);
+        };
+        constexpr uint32_t idesc_dv = ptx::make_idesc_bf16(kBlock, D, true);        // A TMEM, B MN-major
+        constexpr uint32_t idesc_dk = ptx::make_idesc_bf16(kBlock, D, true);        // A K-major, B MN-major
+        constexpr uint32_t idesc_dq = ptx::make_idesc_bf16(kBlock, D, true, true);  // A, B MN-major
+        const uint32_t ds_base = base + L::kDsOff;
+        const uint64_t ds_kmajor = ptx::make_smem_desc(ds_base, 16, 1024);             // dS^T rows = keys
+        const uint64_t ds_mnmajor = ptx::make_smem_desc(ds_base, L::kPanelBytes, 1024);  // dS, M = queries
+        const uint64_t k_mnmajor = ptx::make_smem_desc(base + L::kKOff, L::kPanelBytes, 1024);
+        auto issue_s = [&](int qs) { mma_rows_by_rows<D>(leader, tmem + L::kTmemS, base + L::kKOff, q_addr(qs)); };
+        auto issue_dp = [&](int ds) {
+            mma_rows_by_rows<D>(leader, tmem + L::kTmemDP, base + L::kVOff, do_addr(ds));
+        };
+
+        bool ok = wait_all(kv_full, 0) && nb > 0;
+        if (ok) ok = wait_all(q_full(0), 0);
+        if (ok) {
+            ptx::tc_fence_after_sync();
+            issue_s(0);
+            commit(s_full);
+            ok = wait_all(do_full(0), 0);
+        }
+        if (ok) {
+            ptx::tc_fence_after_sync();
+            issue_dp(0);
+            commit(dp_full);
+        }
+        for (int b = 0; b < nb && ok; ++b) {
+            const int qs = b % kQSlots, ds = b % L::kDoSlots;
+            const uint32_t ph = b & 1;
+            // dV += P^T dO_i: P^T from TMEM (16 queries = 8 columns per step;
+            // queries [64h, 64h + 64) sit at columns [64h, 64h + 32)), dO_i MN-major.
+            ok = wait_all(p_full, ph);
             if (!ok) break;
             ptx::tc_fence_after_sync();
-            uint32_t pp[2][16], ds[2][16];
+            {
+                const uint64_t dod = ptx::make_smem_desc(do_addr(ds), L::kPanelBytes, 1024);
 #pragma unroll
-            for (int ci = 0; ci < 2; ++ci) {
-                const int c0 = h * (kBlock / 2) + ci * 32;
-                uint32_t sv[32], gv[32];
-                ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemS + c0, sv);
-                ptx::tmem_ld32_wait(tmem + lane_addr + L::kTmemDP + c0, gv);
+                for (int ks = 0; ks < kBlock / 16; ++ks)
+                    if (leader)
+                        ptx::mma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + 64 * (ks >> 2) + 8 * (ks & 3),
+                                    dod + ((ks * 16 * 128) >> 4), idesc_dv, (b > 0 || ks > 0) ? 1u : 0u);
+            }
+            commit(do_empty(ds));
+            // S^T(i+1) over P^T(i): issued after dV(i), executed after it
+            if (b + 1 < nb) {
+                ok = wait_all(q_full((b + 1) % kQSlots), ((b + 1) / kQSlots) & 1);
+                if (!ok) break;
+                ptx::tc_fence_after_sync();
+                issue_s((b + 1) % kQSlots);
+                commit(s_full);
+            }
+            ok = wait_all(ds_full, ph);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            // dQ_i = dS K into the dP^T columns (read by the compute warps by now)
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p2[2], d2[2];
+            for (int ks = 0; ks < kBlock / 16; ++ks)
+                if (leader)
+                    ptx::mma_ss(tmem + L::kTmemDP, ds_mnmajor + ((ks * 16 * 128) >> 4),
+                                k_mnmajor + ((ks * 16 * 128) >> 4), idesc_dq, ks > 0 ? 1u : 0u);
+            commit(dq_full);
+            // dK += dS^T Q_i
+            {
+                const uint64_t qd = ptx::make_smem_desc(q_addr(qs), L::kPanelBytes, 1024);
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int qc = c0 + e + u;  // query within the block
-                        const int qrow = i * kBlock + qc;
-                        const bool use = kvalid && qrow < p.n && (!kCausal || key <= qrow);
-                        p2[u] = use ? ptx::ex2(__uint_as_float(sv[e + u]) * p.scale_log2 - lse2_sm[qc]) : 0.f;
-                        d2[u] = p2[u] * (__uint_as_float(gv[e + u]) - dsum_sm[qc]);
-                    }
-                    pp[ci][e >> 1] = ptx::pack_bf16x2(p2[0], p2[1]);
-                    ds[ci][e >> 1] = ptx::pack_bf16x2(d2[0], d2[1]);
+                for (int ks = 0; ks < kBlock / 16; ++ks) {
+                    const uint32_t off = ((ks >> 2) * L::kPanelBytes + (ks & 3) * 32) >> 4;
+                    if (leader)
+                        ptx::mma_ss(tmem + L::kTmemDK, ds_kmajor + off, qd + ((ks * 16 * 128) >> 4), idesc_dk,
+                                    (b > 0 || ks > 0) ? 1u : 0u);
                 }
             }
-            // P^T goes over S^T and dS^T over dP^T: the second warp's results
-            // land on columns the first warp reads, so the pair meets first
-            asm volatile("bar.sync %0, 64;" ::"r"(2 + q4) : "memory");
+            commit(q_empty(qs));
+            commit(ds_free);
+            // dP^T(i+1) once dQ_i has left TMEM
+            if (b + 1 < nb) {
+                ok = wait_all(dq_free, ph);
+                if (!ok) break;
+                ok = wait_all(do_full((b + 1) % L::kDoSlots), ((b + 1) / L::kDoSlots) & 1);
+                if (!ok) break;
+                ptx::tc_fence_after_sync();
+                issue_dp((b + 1) % L::kDoSlots);
+                commit(dp_full);
+            }
+        }
+        commit(done);
+        commit(drain);
+        fa::tc::drain_bar(sync, drain, 0);
+        __syncwarp();
+    } else if (warp < kComputeWarps) {
+        // ------------------------------------------------------------ compute warps
+        // Thread = key row r of the block (TMEM lane); the warp's half h of
+        // the 128 query columns.
+        const int q4 = warp & 3, h = warp >> 2;
+        const int r = q4 * 32 + lane;
+        const int key = kb * kBlock + r;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+        const uint32_t t_s = tmem + lane_addr + L::kTmemS + 64 * h;
+        const uint32_t t_dp = tmem + lane_addr + L::kTmemDP + 64 * h;
+        // this thread's row of panel h of the dS^T tile (128-byte swizzle: 16-byte
+        // chunk c of row r sits at chunk position c ^ (r % 8))
+        uint8_t* ds_row = smem + L::kDsOff + h * L::kPanelBytes + r * 128;
+        const float sl = p.scale_log2;
+        bool ok = true;
+        for (int b = 0; b < nb && ok; ++b) {
+            const int i = i_begin + b;
+            const uint32_t ph = b & 1;
+            const float* lv = vec_ptr(b % kQSlots) + 64 * h;
+            const float* dv = lv + kBlock;
+            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, s_full, ph));
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            float pr[64];
+            {
+                uint32_t sv[64];
+                ptx::tmem_ld64_wait(t_s, sv);
+                const bool diag = kCausal && i == kb;  // mask keys after the query
 #pragma unroll
-            for (int ci = 0; ci < 2; ++ci) {
-                const int c0 = h * (kBlock / 2) + ci * 32;
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemS + c0 / 2, pp[ci]);
-                ptx::tmem_st16(tmem + lane_addr + L::kTmemDP + c0 / 2, ds[ci]);
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(lv + c);
+                    float x0, x1, x2, x3;
+                    ptx::fma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl, sl, l4.x, l4.y);
+                    ptx::fma2(x2, x3, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]), sl, sl, l4.z, l4.w);
+                    pr[c] = ptx::ex2(x0);
+                    pr[c + 1] = ptx::ex2(x1);
+                    pr[c + 2] = ptx::ex2(x2);
+                    pr[c + 3] = ptx::ex2(x3);
+                    if (diag) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (r > 64 * h + c + u) pr[c + u] = 0.f;
+                    }
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) pk[c >> 1] = ptx::pack_bf16x2(pr[c], pr[c + 1]);
+                ptx::tmem_st32(t_s, pk);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(c.p_full());
+            ptx::mbar_arrive(p_full);
+
+            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, dp_full, ph));
+            if (ok && b > 0) ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, ds_free, ph ^ 1));
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t gv[32];
+                ptx::tmem_ld32_wait(t_dp + 32 * half, gv);
+                uint32_t w[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const int cc = 32 * half + c;
+                    const float4 d4 = *reinterpret_cast<const float4*>(dv + cc);
+                    float e0, e1, e2, e3;
+                    ptx::add2(e0, e1, __uint_as_float(gv[c]), __uint_as_float(gv[c + 1]), -d4.x, -d4.y);
+                    ptx::add2(e2, e3, __uint_as_float(gv[c + 2]), __uint_as_float(gv[c + 3]), -d4.z, -d4.w);
+                    ptx::mul2(e0, e1, e0, e1, pr[cc], pr[cc + 1]);
+                    ptx::mul2(e2, e3, e2, e3, pr[cc + 2], pr[cc + 3]);
+                    w[c >> 1] = ptx::pack_bf16x2(e0, e1);
+                    w[(c >> 1) + 1] = ptx::pack_bf16x2(e2, e3);
+                }
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int chunk = 4 * half + v;  // 16-byte chunk (8 queries) of the 128-byte row
+                    *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before_sync();
+            ptx::mbar_arrive(ds_full);
         }
-        if (ok) ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, c.done(), 0));
+        if (ok) ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, done, 0));
         if (ok) {
             ptx::tc_fence_after_sync();
+            const bool kvalid = key < p.n;
             const int64_t off = (static_cast<int64_t>(bh) * p.n + key) * D;
-            store_rows<D>(tmem + lane_addr + L::kTmemAcc0, p.out0 + off, kvalid, 1.f, h * (D / 2));      // dV
-            store_rows<D>(tmem + lane_addr + L::kTmemAcc1, p.out1 + off, kvalid, p.scale, h * (D / 2));  // dK
+            store_rows<D>(tmem + lane_addr + L::kTmemDV, p.dv + off, kvalid, 1.f, h * (D / 2));
+            store_rows<D>(tmem + lane_addr + L::kTmemDK, p.dk + off, kvalid, p.scale, h * (D / 2));
         }
+    } else if (warp >= kDrainWarp0) {
+        // ------------------------------------------------------------ dQ drain
+        // Warp = one lane quarter (32 query rows) of dQ_i.  Columns go from
+        // TMEM to registers 64 at a time; 32 at a time from registers into
+        // this warp's 4 KB staging tile (128-byte swizzle) and on into the fp32
+        // accumulator by a TMA reduce-add.  TMEM is released (dq_free) as soon
+        // as every column is in registers or staged, so dP^T(i+1) can follow.
+        const int q4 = warp & 3;
+        const uint32_t t_dq = tmem + (static_cast<uint32_t>(32 * q4) << 16) + L::kTmemDP;
+        const uint32_t stage = base + L::kStageOff + (warp - kDrainWarp0) * kStageBytes;
+        uint8_t* stage_row = smem + L::kStageOff + (warp - kDrainWarp0) * kStageBytes + lane * 128;
+        auto put = [&](const uint32_t* vals, int c0, int row0, int bhh) {
+            if (lane == 0) ptx::bulk_wait_group_read0();  // the previous reduce has read the tile
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(stage_row + ((c ^ (lane & 7)) << 4)) =
+                    make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::tma_reduce_add_3d(&tm_dq, stage, c0, row0, bhh);
+                ptx::bulk_commit_group();
+            }
+        };
+        bool ok = true;
+        for (int b = 0; b < nb && ok; ++b) {
+            const int row0 = (i_begin + b) * kBlock + 32 * q4;
+            ok = __all_sync(0xffffffffu, fa::tc::wait_bar(sync, dq_full, b & 1));
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
+            uint32_t lo[64];
+            ptx::tmem_ld64_wait(t_dq, lo);
+            if constexpr (D == 64) {
+                ptx::tc_fence_before_sync();
+                ptx::mbar_arrive(dq_free);
+                put(lo, 0, row0, bh);
+                put(lo + 32, 32, row0, bh);
+            } else {
+                put(lo, 0, row0, bh);
+                uint32_t hi[64];
+                ptx::tmem_ld64_wait(t_dq + 64, hi);
+                ptx::tc_fence_before_sync();
+                ptx::mbar_arrive(dq_free);
+                put(lo + 32, 32, row0, bh);
+                put(hi, 64, row0, bh);
+                put(hi + 32, 96, row0, bh);
+            }
+        }
+        if (lane == 0) ptx::bulk_wait_group0();  // every reduce-add has landed
+        __syncwarp();
     }
+
+    // ---------------------------------------------------------------- teardown
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
