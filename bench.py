@@ -24,8 +24,10 @@ zig-zag layout that gives every rank the same causal work).
 `--path backward` measures fa_bwd (dq, dk, dv from the saved lse) on the same
 workload, counting the customary 2.5x the forward's FLOPs.  `--path fp8`
 measures fa_fwd_fp8 (E4M3 Q, K, V, bf16 O) on an E4M3 workload of the same
-shape (default e4m3_b2h32_n8192_d128_causal) against the measured bf16 peak
-times the nominal FP8/BF16 ratio of 2.  `--path decode`
+shape (default e4m3_b2h32_n8192_d128_causal) against an E4M3 cuBLAS GEMM
+timed in the same run (and, beside it, the measured bf16 peak times the
+nominal FP8/BF16 ratio of 2).  `--path peaks` times the bf16 and E4M3
+library GEMMs alone.  `--path decode`
 measures the generation step instead (fa_decode: new queries
 over a resident key/value cache, HBM-bound): the metric is the cache bytes
 read per second, against the measured HBM copy bandwidth.
@@ -68,7 +70,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
-    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward", "ring", "fp8"])
+    ap.add_argument("--path", default="forward", choices=["forward", "decode", "backward", "ring", "fp8", "peaks"])
     ap.add_argument("--ring-chunks", type=int, default=4,
                     help="--path ring on one GPU: sequence chunks emulated one rank after another")
     ap.add_argument("--decode-workload", default=W.DECODE_HEADLINE.name, choices=sorted(W.DECODE_BY_NAME))
@@ -164,6 +166,18 @@ class ClockSampler:
         reasons = sorted({x for r in loaded for x in r["reasons"]})
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": loaded[0]["smax"],
                 "reasons": reasons, "samples": len(loaded)}
+
+
+def add_cycles(line: dict, ms: float) -> None:
+    """Clock-neutral cost of a step beside the timed one: SM cycles per step
+    (ms x the median SM clock sampled under load) and the metric scaled to
+    the maximum SM clock, so runs at different (power-capped) clocks compare."""
+    c = line.get("clocks") or {}
+    mhz, mx = c.get("sm_mhz"), c.get("sm_max_mhz")
+    if mhz:
+        c["sm_cycles_per_step"] = ms * 1e-3 * mhz * 1e6
+        if mx and "value" in line:
+            c["value_at_max_clock"] = line["value"] * mx / mhz
 
 
 def sample_rows_for(w: W.Workload, seconds: float, seed: int):
@@ -307,6 +321,7 @@ def run_ours(a, w: W.Workload):
             else f"fa_fwd_f32_kernel<{w.d},{str(w.causal).lower()}>",
             "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
         line["clocks"] = clocks.summary()
+        add_cycles(line, ms)
         line["gpu_launches"] = a.steps
 
     if "e2e" in legs:
@@ -402,15 +417,19 @@ def run_fp8(a, w: W.Workload):
         peak, peak_sus, _, peak_kind = measured_peaks()
         line["value"] = world * tflops_rank
         line["ms_per_step"] = ms
+        e4m3_peak = gemm_peak_tflops("e4m3", dev)
         line["roofline"] = {
-            "bound": "tensor", "achieved": tflops_rank, "peak": 2 * peak, "unit": "TFLOP/s",
-            "frac": tflops_rank / (2 * peak),
-            "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS) x 2, the nominal FP8/BF16 ratio",
+            "bound": "tensor", "achieved": tflops_rank, "peak": e4m3_peak, "unit": "TFLOP/s",
+            "frac": tflops_rank / e4m3_peak,
+            "peak_kind": "measured here: cuBLAS E4M3 8192^3 (torch._scaled_mm), best of 10",
+            "frac_of_nominal_ratio": tflops_rank / (2 * peak),
+            "nominal_ratio_peak": f"{peak_kind} dense bf16 burst (cuBLAS) x 2, the nominal FP8/BF16 ratio",
             "frac_of_sustained": tflops_rank / (2 * peak_sus),
             "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
             "kernel": f"fa_fwd_e4m3_kernel<{str(w.causal).lower()}>",
             "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
         line["clocks"] = clocks.summary()
+        add_cycles(line, ms)
         line["gpu_launches"] = a.steps
     if "e2e" in legs:
         o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -560,6 +579,7 @@ def run_decode(a, w: W.DecodeWorkload):
                             "kernel": f"fa_decode_mma_kernel<{w.d}>" if esz == 2 else
                             f"fa_decode_kernel<f32,{w.d},{1 if w.nq == 1 else 4}>"}
         line["clocks"] = clocks.summary()
+        add_cycles(line, ms)
         line["gpu_launches"] = a.steps
     if "e2e" in legs:
         # one generation step through the public API: the new tokens' q, k, v
@@ -696,6 +716,7 @@ def run_backward(a, w: W.Workload):
                                     "(three launches); every product runs once on the tensor cores, dQ partials "
                                     "are added into an fp32 buffer by TMA reduce-adds"}
         line["clocks"] = clocks.summary()
+        add_cycles(line, ms)
         line["gpu_launches"] = 3 * a.steps
     if "e2e" in legs:
         o_h = o.cpu().pin_memory()
@@ -810,6 +831,7 @@ def run_ring(a, w: W.Workload):
                          "traffic": None, "kernel": "fa_fwd_bf16_kernel per chunk pair + fa_merge_kernel"},
             "clocks": clocks.summary(),
             "gpu_launches": a.steps * ring_launches_per_rank(chunks, w.causal) * (1 if world > 1 else chunks)}
+    add_cycles(line, ms)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -818,8 +840,52 @@ def run_ring(a, w: W.Workload):
     return 0
 
 
+def gemm_peak_tflops(kind: str, dev, n: int = 8192) -> float:
+    """Best-of-10 TFLOP/s of the library's dense GEMM (cuBLAS via torch) at
+    M = N = K = n: kind "bf16" (torch.matmul) or "e4m3" (torch._scaled_mm,
+    unit fp32 scales, bf16 out), after 3 warm-up runs."""
+    g = torch.Generator(device="cpu").manual_seed(0)
+    a16 = torch.randn(n, n, generator=g).to(dev, torch.bfloat16)
+    b16 = torch.randn(n, n, generator=g).to(dev, torch.bfloat16)
+    if kind == "bf16":
+        fn = lambda: torch.matmul(a16, b16)
+    else:
+        a8 = a16.to(torch.float8_e4m3fn)
+        b8 = b16.to(torch.float8_e4m3fn).t()  # column-major second operand, as _scaled_mm wants
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        fn = lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(3):
+        fn()
+    best = float("inf")
+    for _ in range(10):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e))
+    return 2 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def run_peaks(a):
+    """Dense GEMM throughput of the library routines on this GPU, as roofline
+    denominators: cuBLAS bf16 and E4M3 (see gemm_peak_tflops)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    with ClockSampler(0, enabled=not a.no_clocks) as clocks:
+        out = {kind: gemm_peak_tflops(kind, dev) for kind in ("bf16", "e4m3")}
+    line = {"metric": "dense GEMM peak (library routine)", "unit": "TFLOP/s", "value": out["e4m3"],
+            "config": {"workload": "M=N=K=8192", "bf16_tflops": out["bf16"], "e4m3_tflops": out["e4m3"],
+                       "e4m3_over_bf16": out["e4m3"] / out["bf16"]},
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     a = parse()
+    if a.path == "peaks":
+        return run_peaks(a)
     if a.path == "ring":
         return run_ring(a, W.BY_NAME[a.workload])
     if a.path == "backward":

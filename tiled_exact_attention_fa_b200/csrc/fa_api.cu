@@ -839,7 +839,8 @@ int launch_bwd(DeviceState* st, int slot, const void* q, const void* k, const vo
     float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.vec_bytes);
     float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ws.vec_bytes);
     const int64_t prows = bh * npad;
-    fa::bwd::fa_bwd_prep_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, s>>>(
+    constexpr int64_t kPrepRows = 256 / (D / 8);  // rows per 256-thread block
+    fa::bwd::fa_bwd_prep_kernel<D><<<static_cast<unsigned>((prows + kPrepRows - 1) / kPrepRows), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), lse, lvec, dvec, dq_acc, bh,
         static_cast<int>(n), static_cast<int>(npad));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch of the backward preparation kernel");

@@ -111,31 +111,39 @@ struct Params {
 };
 
 // Per row of every head (padded to whole blocks): D, L, and the fp32 dQ
-// accumulator row set to zero.  One warp per row.
+// accumulator row set to zero.  D / 8 threads per row, 8 elements each
+// (16-byte loads of dO and O, two 16-byte zero stores).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const __nv_bfloat16* dout, const __nv_bfloat16* o,
                                                           const float* lse, float* lvec, float* dvec,
                                                           float* dq_acc, int64_t bh, int n, int npad) {
-    const int64_t prow = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // padded row index
-    const int lane = threadIdx.x & 31;
-    if (prow >= bh * npad) return;
+    constexpr int kPerRow = D / 8;                   // threads per row (a power of two dividing 32)
+    const int64_t prow = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) / kPerRow;  // padded row
+    const int part = threadIdx.x % kPerRow;
+    const bool live = prow < bh * npad;              // (every lane stays for the shuffles below)
     const int64_t head = prow / npad;
     const int r = static_cast<int>(prow - head * npad);
-    constexpr int kPer = D / 32;
     float acc = 0.f;
-    if (r < n) {
+    if (live && r < n) {
         const int64_t row = head * n + r;
-        const __nv_bfloat16* a = dout + row * D + lane * kPer;
-        const __nv_bfloat16* b = o + row * D + lane * kPer;
+        const uint4 a = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
+        const uint4 b = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int e = 0; e < kPer; ++e) acc = fmaf(__bfloat162float(a[e]), __bfloat162float(b[e]), acc);
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        for (int e = 0; e < 4; ++e) {
+            const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[e]));
+            const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[e]));
+            acc = fmaf(af.x, bf.x, acc);
+            acc = fmaf(af.y, bf.y, acc);
+        }
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + prow * D);
 #pragma unroll
-    for (int e = lane; e < D / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane == 0) {
+    for (int off = kPerRow / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (!live) return;
+    float4* z = reinterpret_cast<float4*>(dq_acc + prow * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (part == 0) {
         dvec[prow] = acc;
         lvec[prow] = r < n ? -lse[head * n + r] * kLog2e : -INFINITY;
     }
