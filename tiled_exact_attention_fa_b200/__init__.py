@@ -52,7 +52,6 @@ _SIGNATURES = {
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_version": (ctypes.c_int, []),
     # include/fa_testing.h
-    "fa_test_exp2_poly": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]),
     "fa_test_skip_one_arrival": (ctypes.c_int, []),
 }
 

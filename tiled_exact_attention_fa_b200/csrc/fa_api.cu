@@ -238,34 +238,12 @@ int dispatch(DeviceState* st, const void* q, const void* k, const void* v, void*
              : launch_f32<64, false>(q, k, v, o, lse, bh, N, scale, s);
 }
 
-__global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
-    const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
-    if (i >= n) return;
-    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
-    float y0, y1;
-    fa::ptx::exp2_poly2(y0, y1, x0, x1);
-    y[i] = y0;
-    if (i + 1 < n) y[i + 1] = y1;
-}
-
 }  // namespace
 
 extern "C" {
 
 int fa_test_skip_one_arrival(void) {
     g_skip_one_arrival.store(1);
-    return FA_OK;
-}
-
-int fa_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-    g_last_error.clear();
-    if (n < 0 || (n > 0 && (!x || !y))) return fail(FA_ERR_INVALID_ARGUMENT, "bad exp2 test arguments");
-    if (n == 0) return FA_OK;
-    const int64_t pairs = (n + 1) / 2;
-    const unsigned blocks = static_cast<unsigned>((pairs + 255) / 256);
-    exp2_poly_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "launch of the exp2 test kernel");
     return FA_OK;
 }
 
@@ -1020,7 +998,7 @@ int launch_e4m3(DeviceState* st, const void* q, const void* k, const void* v, vo
     p.base.skip_one_arrival = 0;
     p.o_scale = o_scale;
     const int grid = p.base.num_units < st->sm_count ? p.base.num_units : st->sm_count;
-    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    kernel<<<grid, fa::tc8::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the E4M3 attention kernel");
     return FA_OK;

@@ -57,13 +57,14 @@ namespace tc8 {
 
 using tc::kBlockM;
 using tc::kBlockN;
-using tc::kLoadWarp;
-using tc::kMmaWarp;
 using tc::kSchedDepth;
-using tc::kSoftmaxWarps;
-using tc::kThreads;
 using tc::kTmemCols;
 using tc::kUnitRows;
+
+constexpr int kSoftmaxWarps = 16;      // 8 per query tile
+constexpr int kMmaWarp = 16;
+constexpr int kLoadWarp = 17;
+constexpr int kThreads = 576;
 
 constexpr int D = 128;                 // head dim (one 128-byte row of E4M3)
 constexpr int kSlots = 8;              // K/V ring slots

@@ -398,34 +398,5 @@ __device__ __forceinline__ void add_bf16x2_to_f32(float& acc0, float& acc1, uint
         : "r"(v));
 }
 
-// 2^x for two values on the FMA/ALU pipes instead of the special-function
-// unit.  Range reduction x = j + f with j = round(x), f in [-1/2, 1/2]; a cubic
-// fitted (minimax in relative error, max 7.5e-5 = 2^-13.7, see
-// fit_exp2_poly.py) gives 2^f; 2^j is added to the exponent field.  Inputs
-// below -125 are clamped there (results under 2^-125 are negligible next to
-// the row's running sum, which is at least 1).
-constexpr float kExp2C0 = 0x1.fff692p-1f;
-constexpr float kExp2C1 = 0x1.62f31ap-1f;
-constexpr float kExp2C2 = 0x1.f0de1ap-3f;
-constexpr float kExp2C3 = 0x1.c3f76p-5f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-    // x is clamped to [-125, 127], where round(x) + the exponent of the
-    // polynomial's value stays a normal fp32 exponent: a tiny positive value
-    // below, a huge finite one (>= 2^126) above.
-    x0 = fminf(fmaxf(x0, -125.f), 127.f);
-    x1 = fminf(fmaxf(x1, -125.f), 127.f);
-    float t0, t1, r0, r1, f0, f1, p0, p1;
-    add2(t0, t1, x0, x1, kRoundMagic, kRoundMagic);      // low mantissa bits hold round(x)
-    add2(r0, r1, t0, t1, -kRoundMagic, -kRoundMagic);    // round(x), exact
-    fma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);            // f = x - round(x)
-    fma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
-    fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-    fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 }  // namespace ptx
 }  // namespace fa
