@@ -91,17 +91,18 @@ def kernel_digest(kind: str) -> str:
     return fb.code_digest(fb.KERNEL_SOURCES[kind])
 
 
-def traffic_from_profile(w):
+def traffic_from_profile(w, kind: str | None = None):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
     workload, or None when there is none or the kernel changed since."""
-    path = os.path.join(PROFILE_DIR, f"traffic_{w.name}.json")
+    suffix = "_bwd" if kind == "backward" else ""
+    path = os.path.join(PROFILE_DIR, f"traffic_{w.name}{suffix}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if isinstance(w, W.DecodeWorkload):
+    if kind is None and isinstance(w, W.DecodeWorkload):
         kind = "decode_mma" if w.dtype == torch.bfloat16 else "decode"
-    else:
+    elif kind is None:
         kind = "forward_fp8" if w.dtype == torch.float8_e4m3fn else "forward"
     if d.get("kernel_digest") != kernel_digest(kind):
         return None
@@ -657,6 +658,14 @@ def bwd_cpu_sample(w: W.Workload, seconds: float, seed: int):
     return flops / dt / 1e12, heads, dt, n
 
 
+def bwd_algorithmic_bytes(w: W.Workload) -> int:
+    """Bytes the fused backward kernel must move per launch: Q, K, V, dO read
+    once, dK, dV written once, and the fp32 dQ accumulator written once (its
+    reduce-adds otherwise stay in L2)."""
+    t = w.B * w.H * w.N * w.d
+    return 4 * t * 2 + 2 * t * 2 + t * 4
+
+
 def run_backward(a, w: W.Workload):
     import tiled_exact_attention_fa_b200 as fa
 
@@ -714,7 +723,9 @@ def run_backward(a, w: W.Workload):
         line["pct_of_bf16_peak"] = 100.0 * tf / peak
         line["roofline"] = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                             "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)", "frac_of_sustained": tf / peak_sus,
-                            "traffic": None, "kernel": "fa_bwd_kernel (+ fa_bwd_prep_kernel, fa_bwd_dq_convert_kernel)",
+                            "traffic": traffic_from_profile(w, "backward"),
+                            "algorithmic_bytes": bwd_algorithmic_bytes(w),
+                            "kernel": "fa_bwd_kernel (+ fa_bwd_prep_kernel, fa_bwd_dq_convert_kernel)",
                             "note": "achieved counts 10*N^2*d (halved for causal) over the whole backward step "
                                     "(three launches); every product runs once on the tensor cores, dQ partials "
                                     "are added into an fp32 buffer by TMA reduce-adds"}

@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "decode": ["fa_decode.cuh", "sm100_ptx.cuh"],
     "decode_mma": ["fa_decode_mma.cuh", "fa_decode.cuh", "sm100_ptx.cuh"],
     "forward_fp8": ["fa_fwd_fp8_tc.cuh", "fa_fwd_tc.cuh", "sm100_ptx.cuh"],
+    "backward": ["fa_bwd_tc.cuh", "fa_fwd_tc.cuh", "sm100_ptx.cuh"],
 }
 
 
