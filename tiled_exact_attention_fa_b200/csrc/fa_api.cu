@@ -135,11 +135,12 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
         std::lock_guard<std::mutex> lock(g_mu);
         st->smem_raised[slot] = true;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     int rc;
     if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&to, o, bh, n, D)) != FA_OK) return rc;
 
     fa::tc::Params p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -154,7 +155,7 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
-    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the bf16 attention kernel");
     return FA_OK;
@@ -368,11 +369,12 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
         std::lock_guard<std::mutex> lock(g_mu);
         st->smem_raised[slot] = true;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     int rc;
     if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
     if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&to, o, bh, n, D)) != FA_OK) return rc;
     // The array keeps the previous call's contents: the queue counters must
     // start at zero, so clear them in stream order.  The status word is left
     // alone, so that a timeout stays visible until fa_noalloc_check_status.
@@ -392,7 +394,7 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
-    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the bf16 attention kernel (no-alloc)");
     return FA_OK;

@@ -27,10 +27,14 @@
 //     (t = 0, 1), two warps per TMEM lane quarter, so a quad of threads owns
 //     two rows: they read S_t from TMEM, update m and l, write P_t (bf16)
 //     back over S_t, rescale O_t in TMEM when a block outgrows the running
-//     max, and at the end normalise O_t and store O and lse.  While one
-//     tile's warps exponentiate, the tensor core works on the other tile.
-//     At d = 128 the exponentials on the special-function unit take about as
-//     long as the tile's MMAs, so they are the co-limit of the kernel.
+//     max, and at the end of a unit write lse, normalise O_t by l and lay it
+//     out in a shared-memory staging tile.  While one tile's warps
+//     exponentiate, the tensor core works on the other tile.  At d = 128 the
+//     exponentials on the special-function unit take about as long as the
+//     tile's MMAs, so they are the co-limit of the kernel;
+//   * warp 18 stores each staged O tile with a TMA tensor store (rows past
+//     N are not written) and frees the staging tile once the store has read
+//     it, so no softmax thread issues the 128 row-strided stores of a tile.
 //   * Causal: KV blocks entirely above the diagonal are never loaded or
 //     multiplied; only the diagonal block is masked.
 //
@@ -62,7 +66,8 @@ constexpr int kUnitRows = kBlockM * kTilesPerUnit;
 constexpr int kSoftmaxWarps = 16;       // 8 per query tile
 constexpr int kMmaWarp = 16;
 constexpr int kLoadWarp = 17;
-constexpr int kThreads = 576;
+constexpr int kEpiWarp = 18;            // stores each finished tile of O with TMA
+constexpr int kThreads = 608;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kStaleMaxBound = 1048576.0f;  // 2^20: largest p accepted against a stale running max
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz
@@ -80,14 +85,17 @@ struct Layout {
     static constexpr int kRingOff = kQOff + kTilesPerUnit * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2],
-    //           sched_full[kSchedDepth], sched_empty[kSchedDepth], drain, pair[2][4]
-    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1 + 8;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base, abort flag, unit ring
-    static constexpr int kInvLOff = (kMiscOff + 8 + 4 * kSchedDepth + 15) & ~15;  // float[2][128]
-    static constexpr int kBytes = kInvLOff + 2 * kBlockM * 4;
+    //           sched_full[kSchedDepth], sched_empty[kSchedDepth], drain, pair[2][4],
+    //           stage_full[2], stage_free
+    static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1 + 8 + 3;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base, abort flag, unit ring, tile coordinates
+    static constexpr int kInvLOff = (kMiscOff + 8 + 4 * kSchedDepth + 16 + 15) & ~15;  // float[2][128]
+    static constexpr int kStageOff = (kInvLOff + 2 * kBlockM * 4 + 1023) & ~1023;   // one 128 x D bf16 O tile
+    static constexpr int kBytes = kStageOff + kTileBytes;
     static constexpr int kSmemBytes = kBytes + 1024;           // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
     static constexpr uint32_t kTmemO = 256;
+    static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct Params {
@@ -196,7 +204,8 @@ template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, const Params p) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_addr(smem_raw);
@@ -220,6 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t drain = bar0 + 8u * (10 + 2 * L::kSlots + 2 * kSchedDepth);
     // the two softmax warps of tile t that share TMEM lane quarter q meet here in the epilogue
     auto pair_bar = [&](int t, int q) { return bar0 + 8u * (11 + 2 * L::kSlots + 2 * kSchedDepth + 4 * t + q); };
+    // the O staging tile: filled by tile t's softmax warps (stage_full(t)),
+    // stored by the epilogue warp, free again once the store has read it
+    auto stage_full = [&](int t) { return bar0 + 8u * (19 + 2 * L::kSlots + 2 * kSchedDepth + t); };
+    const uint32_t stage_free = bar0 + 8u * (21 + 2 * L::kSlots + 2 * kSchedDepth);
+    volatile int* stage_coord = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8 + 4 * kSchedDepth);  // [t][bh, row0]
 
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -241,8 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < kSchedDepth; ++i) {
             ptx::mbar_init(sched_full(i), 1);
-            ptx::mbar_init(sched_empty(i), 1 + kSoftmaxWarps);
+            ptx::mbar_init(sched_empty(i), 2 + kSoftmaxWarps);
         }
+        ptx::mbar_init(stage_full(0), 32 * (kSoftmaxWarps / 2));
+        ptx::mbar_init(stage_full(1), 32 * (kSoftmaxWarps / 2));
+        ptx::mbar_init(stage_free, 1);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -251,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_alloc(ptx::smem_addr(tmem_base_ptr), kTmemCols);
         ptx::tmem_relinquish();
     }
+    if (warp == kEpiWarp && lane == 0) ptx::prefetch_tmap(&tm_o);
     if (warp == kLoadWarp && lane == 0) {
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
@@ -465,6 +483,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(drain);
         drain_bar(sync, drain, 0);
         __syncwarp();
+    } else if (warp == kEpiWarp) {
+        // ------------------------------------------------------------ epilogue
+        // For each unit, tile 0's then tile 1's O arrive in the staging tile;
+        // one lane stores it with TMA (rows past N are not written) and, once
+        // the store has read shared memory, frees the tile for the next one.
+        bool ok = true;
+        uint32_t uses = 0;
+        for (uint32_t it = 0; ok; ++it) {
+            const int rs = it % kSchedDepth;
+            ok = __all_sync(0xffffffffu, wait_bar(sync, sched_full(rs), (it / kSchedDepth) & 1));
+            if (!ok) break;
+            const int u = unit_ring[rs];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(sched_empty(rs));
+            if (u < 0) break;
+            for (int t = 0; t < 2 && ok; ++t, ++uses) {
+                ok = __all_sync(0xffffffffu, wait_bar(sync, stage_full(t), it & 1));
+                if (!ok) break;
+                if (lane == 0) {
+                    const int bh = stage_coord[2 * t], row0 = stage_coord[2 * t + 1];
+                    for (int hh = 0; hh < L::kHalves; ++hh)
+                        ptx::tma_store_3d(&tm_o, base + L::kStageOff + hh * L::kPanelBytes, hh * 64, row0, bh);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read0();
+                    ptx::mbar_arrive(stage_free);
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) ptx::bulk_wait_group0();  // every store has landed
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax warps
         // Warps 0-7 serve query tile 0 and warps 8-15 tile 1.  The two warps
@@ -487,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* inv_l_sm = reinterpret_cast<float*>(smem + L::kInvLOff) + t * kBlockM;
         const float sl = p.scale_log2;
         uint32_t s_phase = 0, o_phase = 0, pair_phase = 0;
+        uint32_t units = 0;  // units this warp has finished (for the staging tile's turn)
         bool ok = true;
 
         for (uint32_t it = 0; ok; ++it) {
@@ -659,12 +709,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, wait_bar(sync, pair_bar(t, q), pair_phase));
             if (!ok) break;
             pair_phase ^= 1;
-            // O = O_acc / l, written once: this warp stores columns
-            // [D/2 h, D/2 (h+1)) of the quarter's 32 rows, one row per thread.
-            const int row = tile_row0 + 32 * q + lane;
-            const float inv_l = inv_l_sm[32 * q + lane];
-            const bool valid = row < p.n;
-            __nv_bfloat16* orow_g = p.o + (static_cast<int64_t>(w.bh) * p.n + row) * D + (D / 2) * h;
+            // O = O_acc / l, written once: this warp converts columns
+            // [D/2 h, D/2 (h+1)) of the quarter's 32 rows (one row per thread)
+            // into the staging tile, laid out as the TMA store's 128-byte-
+            // swizzled box (64-column panels; 16-byte chunk c of row r at
+            // chunk position c ^ (r % 8)); the epilogue warp stores it.
+            // Turn of the staging tile: tile 0's unit k follows tile 1's unit
+            // k - 1, tile 1's follows tile 0's of the same unit.
+            if (units > 0 || t == 1) {
+                const uint32_t turn = 2 * units + static_cast<uint32_t>(t) - 1;
+                ok = __all_sync(0xffffffffu, wait_bar(sync, stage_free, turn & 1));
+                if (!ok) break;
+            }
+            const int rloc = 32 * q + lane;  // row in the tile
+            const float inv_l = inv_l_sm[rloc];
+            uint8_t* srow = smem + L::kStageOff + ((D / 2) * h / 64) * L::kPanelBytes + rloc * 128;
+            const int chunk0 = ((D / 2) * h % 64) / 8;  // first 16-byte chunk of this warp's columns
 #pragma unroll
             for (int c0 = 0; c0 < D / 2; c0 += 32) {
                 uint32_t acc[32];
@@ -674,15 +734,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 32; c += 2)
                     packed[c >> 1] = ptx::pack_bf16x2(__uint_as_float(acc[c]) * inv_l,
                                                       __uint_as_float(acc[c + 1]) * inv_l);
-                if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow_g + c0);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                            packed[4 * v + 3]);
+                for (int v = 0; v < 4; ++v) {
+                    const int chunk = chunk0 + c0 / 8 + v;
+                    *reinterpret_cast<uint4*>(srow + ((chunk ^ (rloc & 7)) << 4)) =
+                        make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                 }
             }
+            if (warp == 8 * t && lane == 0) {
+                stage_coord[2 * t] = w.bh;
+                stage_coord[2 * t + 1] = tile_row0;
+            }
+            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before_sync();
+            ptx::mbar_arrive(stage_full(t));
+            ++units;
         }
     }
 

@@ -107,6 +107,15 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32
         "r"(src), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 3-D tiled store shared -> global (the tile at `src` laid out as the
+// tensor map's box); rows past the tensor's end are not written.
+// Completion is tracked by the bulk-group mechanism.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk group has finished READING its shared-memory source.
 __device__ __forceinline__ void bulk_wait_group_read0() {
