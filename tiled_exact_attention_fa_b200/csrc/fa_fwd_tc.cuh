@@ -411,34 +411,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             return __all_sync(0xffffffffu, wait_bar(sync, bar, parity));
         };
 
-        for (uint32_t it = 0; ok; ++it) {
+        // Unit `it` from the scheduling ring (-1: the queue is empty).
+        auto fetch_unit = [&](uint32_t it, int& u) {
             const int rs = it % kSchedDepth;
-            ok = wait_all(sched_full(rs), (it / kSchedDepth) & 1);
-            if (!ok) break;
-            const int u = unit_ring[rs];
+            if (!wait_all(sched_full(rs), (it / kSchedDepth) & 1)) return false;
+            u = unit_ring[rs];
             __syncwarp();
             if (leader) ptx::mbar_arrive(sched_empty(rs));
-            if (u < 0) break;
-
-            const Unit w = decode_unit(u, p, kCausal);
-            const int n0 = num_kv_blocks(p, w.qb, 0, kCausal);
-            const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
-            ok = wait_all(q_full(0), it & 1) && wait_all(q_full(1), it & 1);
-            if (!ok) break;
-            int sk, sv;
-            uint32_t pk, pv;
+            return true;
+        };
+        // S_0(0) of a unit: Q_0 of that unit and its first K block.
+        int sk = 0, sv = 0;
+        uint32_t pk = 0, pv = 0;
+        auto first_s0 = [&](uint32_t it, int n0) {
+            if (!wait_all(q_full(0), it & 1)) return false;
             next_slot(sk, pk);
-            ok = wait_all(kv_full(sk), pk);
-            if (!ok) break;
+            if (!wait_all(kv_full(sk), pk)) return false;
             ptx::tc_fence_after_sync();
             issue_s(0, sk);
             commit(s_full(0));
             if (n0 == 1) commit(q_empty(0));
+            return true;
+        };
+
+        int u = -1;
+        ok = fetch_unit(0, u);
+        bool s0_issued = false;  // S_0(0) of unit `it` went out during the previous unit
+        for (uint32_t it = 0; ok && u >= 0; ++it) {
+            const Unit w = decode_unit(u, p, kCausal);
+            const int n0 = num_kv_blocks(p, w.qb, 0, kCausal);
+            const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
+            if (!s0_issued) {
+                ok = first_s0(it, n0);
+                if (!ok) break;
+            }
+            s0_issued = false;
+            ok = wait_all(q_full(1), it & 1);
+            if (!ok) break;
+            ptx::tc_fence_after_sync();
             issue_s(1, sk);
             commit(s_full(1));
             if (n1 == 1) commit(q_empty(1));
             commit(kv_empty(sk));
 
+            int next_u = -1;
+            bool fetched = false;
             for (int j = 0; j < n1 && ok; ++j) {
                 // V_j and K_{j+1} are waited for before P_0(j), so that PV_0(j)
                 // and S_0(j+1) go to the tensor core back to back.
@@ -464,6 +481,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     commit(s_full(0));
                     if (j + 1 == n0 - 1) commit(q_empty(0));
                 }
+                if (!more) {
+                    // Tile 0 is done with this unit: start the next unit's
+                    // tile 0 now, so its warps find S_0(0) ready after their
+                    // epilogue instead of waiting for tile 1's last block.
+                    // (The ring holds this unit's last V, then the next
+                    // unit's first K.)
+                    ok = fetch_unit(it + 1, next_u);
+                    if (!ok) break;
+                    fetched = true;
+                    if (next_u >= 0) {
+                        const Unit wn = decode_unit(next_u, p, kCausal);
+                        ok = first_s0(it + 1, num_kv_blocks(p, wn.qb, 0, kCausal));
+                        if (!ok) break;
+                        s0_issued = true;
+                    }
+                }
                 ok = wait_all(p_full(1), p_phase[1]);
                 if (!ok) break;
                 p_phase[1] ^= 1;
@@ -478,6 +511,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     commit(kv_empty(sk));
                 }
             }
+            if (!ok) break;
+            if (!fetched) {
+                ok = fetch_unit(it + 1, next_u);
+                if (!ok) break;
+            }
+            u = next_u;
         }
         // Drain: all issued MMAs complete before TMEM is released.
         commit(drain);
