@@ -638,11 +638,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // this thread's share of both row sums.
                 uint32_t pk[32];
                 float a[2][2], b[2][2];
-                auto exponentiate = [&](const float (&neg_m)[2]) {
+                // chunks [k0, k1) of the block; a and b accumulate
+                auto exponentiate_chunks = [&](const float (&neg_m)[2], int k0, int k1) {
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) a[r][0] = a[r][1] = b[r][0] = b[r][1] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
+                    for (int k = k0; k < k1; ++k) {
 #pragma unroll
                         for (int r = 0; r < 2; ++r) {
                             float x0, x1, p0, p1;
@@ -656,6 +655,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 };
+                auto exponentiate = [&](const float (&neg_m)[2]) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) a[r][0] = a[r][1] = b[r][0] = b[r][1] = 0.f;
+                    exponentiate_chunks(neg_m, 0, 16);
+                };
                 auto neg_of = [](float m) { return (m == -INFINITY) ? 0.f : -m; };
 
                 // Online softmax.  The first block of a unit sets the running
@@ -666,10 +670,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // everything seen so far -- the block is redone against its
                 // exact max and O and l are rescaled.  O and l always share the
                 // same m, so the result does not depend on how stale m is.
-                load_scores();
+                // Causal instantiation, unmasked later blocks: the second
+                // half of the block's columns loads while the first half is
+                // exponentiated (no TMEM store is issued in between).  The
+                // non-causal instantiation keeps one load at the top: with the
+                // split the compiler spills there and it measured slower.
+                if constexpr (!kCausal) load_scores();
                 float alpha[2] = {1.f, 1.f};
                 bool rescale_o = false;
                 if (j == 0) {
+                    if constexpr (kCausal) load_scores();
                     float mx[2];
                     block_max(mx);
                     m_run[0] = mx[0];
@@ -678,7 +688,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     exponentiate(nm);
                 } else {
                     const float nm[2] = {neg_of(m_run[0]), neg_of(m_run[1])};
-                    exponentiate(nm);
+                    if (!kCausal || need_mask) {
+                        if constexpr (kCausal) load_scores();
+                        exponentiate(nm);
+                    } else {
+                        uint32_t(&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+                        uint32_t(&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+                        ptx::tmem_ld16x256b_x8_wait(tmem_s, lo);
+                        ptx::tmem_ld16x256b_x8(tmem_s + 64, hi);
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) a[r][0] = a[r][1] = b[r][0] = b[r][1] = 0.f;
+                        exponentiate_chunks(nm, 0, 8);
+                        ptx::tmem_wait_ld(hi);
+                        exponentiate_chunks(nm, 8, 16);
+                    }
                     const bool big = (a[0][0] + a[0][1] > kStaleMaxBound) || (a[1][0] + a[1][1] > kStaleMaxBound);
                     if (__any_sync(0xffffffffu, big)) {
                         load_scores();  // P has not been stored: S is still in TMEM

@@ -280,6 +280,28 @@ __device__ __forceinline__ void tmem_ld16x256b_x16_wait(uint32_t taddr, uint32_t
         : "r"(taddr)
         : "memory");
 }
+// .16x256b over 64 columns (32 registers).  The first form waits; the second
+// only issues the load, whose registers are valid after tmem_wait_ld(r) --
+// which names them as operands, so the compiler cannot read them earlier.
+__device__ __forceinline__ void tmem_ld16x256b_x8_wait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_ld16x256b_x4_wait(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
@@ -290,6 +312,15 @@ __device__ __forceinline__ void tmem_ld16x256b_x4_wait(uint32_t taddr, uint32_t 
         : "memory");
 }
 #undef FA_R8
+
+#define FA_RW8(b) "+r"(r[b + 0]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), \
+                  "+r"(r[b + 4]), "+r"(r[b + 5]), "+r"(r[b + 6]), "+r"(r[b + 7])
+// Wait for this thread's outstanding TMEM loads; `r` are the registers of the
+// load issued last (they may be read only after this).
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : FA_RW8(0), FA_RW8(8), FA_RW8(16), FA_RW8(24) : : "memory");
+}
+#undef FA_RW8
 
 #define FA_W8(b) "r"(r[b + 0]), "r"(r[b + 1]), "r"(r[b + 2]), "r"(r[b + 3]), \
                  "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
