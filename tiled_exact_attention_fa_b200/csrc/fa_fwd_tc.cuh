@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(q_full(t), 1);
             ptx::mbar_init(q_empty(t), 1);
             ptx::mbar_init(s_full(t), 1);
-            ptx::mbar_init(p_full(t), 32 * (kSoftmaxWarps / 2));
+            ptx::mbar_init(p_full(t), kSoftmaxWarps / 2);  // one arrival per warp
             for (int q = 0; q < 4; ++q) ptx::mbar_init(pair_bar(t, q), 64);
             ptx::mbar_init(o_full(t), 1);
         }
@@ -739,9 +739,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::tmem_st16x256b_x4(tmem_o + c0, ov);
                     }
                 }
+                // Every lane's P is in TMEM (its own wait and fence), the warp
+                // meets, and one lane arrives: 8 arrivals per block instead
+                // of 256 on the barrier the MMA warp is waiting on.
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before_sync();
-                ptx::mbar_arrive(p_full(t));
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(p_full(t));
             }
             if (!ok) break;
 
