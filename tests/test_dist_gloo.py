@@ -1,5 +1,6 @@
-"""Multi-rank host logic on CPU with the gloo backend (world size 2): head
-sharding, max-over-ranks timing and the all-gather of per-rank results."""
+"""Multi-rank host logic on CPU with the gloo backend (world sizes 2 to 4):
+head sharding, max-over-ranks timing and the all-gather of per-rank results,
+including uneven shards and a rank that holds no head."""
 import os
 import socket
 
@@ -16,14 +17,14 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, total_bh=7):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     try:
         fdist.init("gloo", timeout_s=60)
         # each rank "took" a different time; the job time is the max
         t = fdist.max_over_ranks(1.5 + rank)
-        total_bh, N, d = 7, 5, 3
+        N, d = 5, 3
         a, b = fdist.shard_range(total_bh, rank, world)
         o_full = torch.arange(total_bh * N * d, dtype=torch.float32).view(total_bh, N, d)
         l_full = torch.arange(total_bh * N, dtype=torch.float32).view(total_bh, N)
@@ -37,19 +38,21 @@ def _worker(rank, world, port, q):
             torch.distributed.destroy_process_group()
 
 
-def test_two_ranks_gloo():
+@pytest.mark.parametrize("world,total_bh", [(2, 7), (3, 7), (4, 3)])
+def test_ranks_gloo(world, total_bh):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, total_bh)) for r in range(world)]
     for p in procs:
         p.start()
     results = sorted(q.get(timeout=120) for _ in procs)
     for p in procs:
         p.join(timeout=60)
-    assert [r[1] for r in results] == [2.5, 2.5], results
+    slowest = 1.5 + (world - 1)
+    assert [r[1] for r in results] == [slowest] * world, results
     assert all(r[2] and r[3] for r in results), results
-    assert [r[4] for r in results] == [(0, 4), (4, 7)]
+    assert [r[4] for r in results] == [fdist.shard_range(total_bh, r, world) for r in range(world)]
 
 
 @pytest.mark.parametrize("total,world", [(7, 2), (64, 8), (3, 4), (2048, 3)])
