@@ -169,14 +169,29 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(loaded)}
 
 
+def add_in_kernel_clock(line: dict, rec: dict, steps: int) -> None:
+    """The SM clock the forward kernels themselves saw over the timed steps
+    (each CTA's clock64 cycles over its global-timer nanoseconds, summed over
+    CTAs): nvidia-smi samples every 200 ms, mostly between bursts, and reads
+    the idle boost clock, while the kernel runs power-limited below it."""
+    if not rec.get("ctas"):
+        return
+    c = line.setdefault("clocks", {})
+    c["in_kernel_sm_mhz"] = rec["sm_mhz"]
+    c["in_kernel_cycles_per_launch"] = rec["cycles_per_cta"]
+    c["in_kernel_ctas_per_launch"] = rec["ctas"] / steps
+
+
 def add_cycles(line: dict, ms: float) -> None:
     """Clock-neutral cost of a step beside the timed one: SM cycles per step
-    (ms x the median SM clock sampled under load) and the metric scaled to
-    the maximum SM clock, so runs at different (power-capped) clocks compare."""
+    (ms x the SM clock: the one the kernel measured itself where it records
+    it, else the median sampled under load) and the metric scaled to the
+    maximum SM clock, so runs at different (power-capped) clocks compare."""
     c = line.get("clocks") or {}
-    mhz, mx = c.get("sm_mhz"), c.get("sm_max_mhz")
+    mhz, mx = c.get("in_kernel_sm_mhz") or c.get("sm_mhz"), c.get("sm_max_mhz")
     if mhz:
         c["sm_cycles_per_step"] = ms * 1e-3 * mhz * 1e6
+        c["cycles_clock"] = "in-kernel" if c.get("in_kernel_sm_mhz") else "nvidia-smi median"
         if mx and "value" in line:
             c["value_at_max_clock"] = line["value"] * mx / mhz
 
@@ -296,6 +311,7 @@ def run_ours(a, w: W.Workload):
     elapsed_ms = None
     if "kernel" in legs:
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa.clock_record(reset=True)
         with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
             fdist.barrier(dev)
             torch.cuda.synchronize(dev)
@@ -306,6 +322,7 @@ def run_ours(a, w: W.Workload):
             torch.cuda.synchronize(dev)
             fdist.barrier(dev)
         fa.check_device_status()
+        in_kernel = fa.clock_record(reset=True)
         elapsed_ms = fdist.max_over_ranks(start.elapsed_time(end), dev)
         ms = elapsed_ms / a.steps
         tflops_rank = flops / (ms * 1e-3) / 1e12
@@ -322,6 +339,7 @@ def run_ours(a, w: W.Workload):
             else f"fa_fwd_f32_kernel<{w.d},{str(w.causal).lower()}>",
             "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
         line["clocks"] = clocks.summary()
+        add_in_kernel_clock(line, in_kernel, a.steps)
         add_cycles(line, ms)
         line["gpu_launches"] = a.steps
 
@@ -403,6 +421,7 @@ def run_fp8(a, w: W.Workload):
         "flop_per_step": flops}
     if "kernel" in legs:
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa.clock_record(reset=True)
         with ClockSampler(local_rank, enabled=not a.no_clocks) as clocks:
             fdist.barrier(dev)
             torch.cuda.synchronize(dev)
@@ -413,6 +432,7 @@ def run_fp8(a, w: W.Workload):
             torch.cuda.synchronize(dev)
             fdist.barrier(dev)
         fa.check_device_status()
+        in_kernel = fa.clock_record(reset=True)
         ms = fdist.max_over_ranks(start.elapsed_time(end), dev) / a.steps
         tflops_rank = flops / (ms * 1e-3) / 1e12
         peak, peak_sus, _, peak_kind = measured_peaks()
@@ -430,6 +450,7 @@ def run_fp8(a, w: W.Workload):
             "kernel": f"fa_fwd_e4m3_kernel<{str(w.causal).lower()}>",
             "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
         line["clocks"] = clocks.summary()
+        add_in_kernel_clock(line, in_kernel, a.steps)
         add_cycles(line, ms)
         line["gpu_launches"] = a.steps
     if "e2e" in legs:

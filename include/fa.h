@@ -300,6 +300,23 @@ int fa_merge(const void* o_parts, const float* lse_parts, int64_t parts, int64_t
  */
 int fa_check_device_status(void* stream);
 
+/*
+ * fa_clock_record -- a measurement aid, not part of the attention result:
+ * how fast the SM clock ran while the persistent forward kernels (fa_fwd on
+ * bf16, fa_fwd_fp8; not fa_fwd_noalloc) ran on the current device.  Each CTA
+ * of those kernels adds, when it ends, the SM cycles it ran (clock64), the
+ * global-timer nanoseconds it ran and 1 to three device counters.  This call
+ * synchronises `stream`, then writes the counters to out[0] (cycles),
+ * out[1] (nanoseconds) and out[2] (CTAs), and clears them when `reset` is
+ * non-zero.  out[0] / out[1] is the clock in GHz averaged over the kernels'
+ * running time; out[0] / out[2] the cycles of an average CTA, i.e. of a
+ * launch when every CTA runs to the end.  Launches on other streams that are
+ * still running may or may not be counted yet.
+ *   out   host, int64_t[3], written by the call.
+ * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (out NULL) or FA_ERR_CUDA.
+ */
+int fa_clock_record(void* stream, int reset, int64_t* out);
+
 /* fa_status_string -- static, never-NULL description of a status code. */
 const char* fa_status_string(int status);
 

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "fa_merge": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fa_clock_record": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]),
     "fa_noalloc_check_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_error": (ctypes.c_char_p, []),
@@ -335,3 +336,16 @@ def check_device_status(stream: torch.cuda.Stream | None = None) -> None:
     """Synchronise and raise FaError(FA_ERR_DEVICE_TIMEOUT) if a kernel gave up on a wait."""
     s = (stream or torch.cuda.current_stream()).cuda_stream
     _check(int(library().fa_check_device_status(s)))
+
+
+def clock_record(reset: bool = True, stream: torch.cuda.Stream | None = None) -> dict:
+    """SM clock seen by the persistent forward kernels since the last reset
+    (synchronises `stream`): summed CTA cycles and timer nanoseconds, the CTA
+    count, the average clock in MHz and the cycles of an average CTA."""
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    out = (ctypes.c_int64 * 3)()
+    _check(int(library().fa_clock_record(s, int(reset), out)))
+    cycles, ns, ctas = int(out[0]), int(out[1]), int(out[2])
+    return {"cycles": cycles, "ns": ns, "ctas": ctas,
+            "sm_mhz": 1e3 * cycles / ns if ns else None,
+            "cycles_per_cta": cycles / ctas if ctas else None}

@@ -42,7 +42,8 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 // Per-device state created on the first call that runs on that device and
 // kept until process exit: a small device workspace holding the status word
-// written by kernels that give up on a bounded wait, followed by the work
+// written by kernels that give up on a bounded wait, the forward kernels'
+// clock record (SM cycles, timer nanoseconds, CTAs), followed by the work
 // queues of the persistent kernel (two counters each, returned to zero by the
 // last CTA of every launch); the SM count for the persistent grid; and
 // whether the kernels' shared memory limits were raised.  Successive launches
@@ -50,11 +51,14 @@ int cuda_fail(cudaError_t e, const char* what) {
 // different streams) use different counters unless more than kQueues of them
 // are in flight at once.
 constexpr int kQueues = 1024;
-constexpr size_t kWorkspaceBytes = 16 + kQueues * 2 * sizeof(unsigned);
+constexpr size_t kClockOffset = 16;  // three 64-bit counters
+constexpr size_t kQueueOffset = 48;
+constexpr size_t kWorkspaceBytes = kQueueOffset + kQueues * 2 * sizeof(unsigned);
 
 struct DeviceState {
     bool ready = false;
     int* status = nullptr;
+    unsigned long long* clock = nullptr;
     unsigned* queues = nullptr;
     std::atomic<unsigned> next_queue{0};
     int sm_count = 0;
@@ -97,7 +101,8 @@ int device_state(DeviceState** out) {
         if ((e = cudaMalloc(&ws, kWorkspaceBytes)) != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
         if ((e = cudaMemset(ws, 0, kWorkspaceBytes)) != cudaSuccess) return cuda_fail(e, "cudaMemset(workspace)");
         s.status = static_cast<int*>(ws);
-        s.queues = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + 16);
+        s.clock = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kClockOffset);
+        s.queues = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kQueueOffset);
         s.ready = true;
     }
     *out = &s;
@@ -154,6 +159,7 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     p.num_units = p.bh * p.num_qblocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
+    p.clock = st->clock;
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
     kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     cudaError_t e = cudaGetLastError();
@@ -291,6 +297,23 @@ int fa_check_device_status(void* stream) {
     return FA_OK;
 }
 
+int fa_clock_record(void* stream, int reset, int64_t* out) {
+    g_last_error.clear();
+    if (!out) return fail(FA_ERR_INVALID_ARGUMENT, "out is null");
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned long long h[3] = {0, 0, 0};
+    if ((e = cudaMemcpy(h, st->clock, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpy(clock record)");
+    for (int i = 0; i < 3; ++i) out[i] = static_cast<int64_t>(h[i]);
+    if (reset && (e = cudaMemset(st->clock, 0, sizeof(h))) != cudaSuccess)
+        return cuda_fail(e, "cudaMemset(clock record)");
+    return FA_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -393,6 +416,7 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     p.num_units = p.bh * p.num_qblocks;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
+    p.clock = nullptr;  // nothing of the shared workspace is touched here
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
     kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     e = cudaGetLastError();
@@ -998,6 +1022,7 @@ int launch_e4m3(DeviceState* st, const void* q, const void* k, const void* v, vo
     p.base.num_units = p.base.bh * p.base.num_qblocks;
     p.base.scale_log2 = static_cast<float>(scale_qk * 1.4426950408889634);
     p.base.skip_one_arrival = 0;
+    p.base.clock = st->clock;
     p.o_scale = o_scale;
     const int grid = p.base.num_units < st->sm_count ? p.base.num_units : st->sm_count;
     kernel<<<grid, fa::tc8::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);

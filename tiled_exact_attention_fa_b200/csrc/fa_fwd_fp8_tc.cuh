@@ -84,7 +84,8 @@ struct Layout {
     static constexpr int kBarSchedEmpty = kBarSchedFull + kSchedDepth, kBarDrain = kBarSchedEmpty + kSchedDepth;
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag, unit ring
-    static constexpr int kBytes = kMiscOff + 8 + 4 * kSchedDepth;
+    static constexpr int kClockOff = (kMiscOff + 8 + 4 * kSchedDepth + 7) & ~7;  // int64[2]: start clock, timer
+    static constexpr int kBytes = kClockOff + 16;
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
     static constexpr uint32_t kTmemO = 256;
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw);
+    tc::clock_start(p, smem + L::kClockOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -688,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
+    tc::clock_end(p, smem + L::kClockOff);
 }
 
 }  // namespace tc8

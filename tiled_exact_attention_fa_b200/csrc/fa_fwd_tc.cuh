@@ -90,7 +90,8 @@ struct Layout {
     static constexpr int kNumBars = 2 + 2 + kSlots + kSlots + 2 + 2 + 2 + 2 * kSchedDepth + 1 + 8 + 3;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;    // tmem base, abort flag, unit ring, tile coordinates
     static constexpr int kInvLOff = (kMiscOff + 8 + 4 * kSchedDepth + 16 + 15) & ~15;  // float[2][128]
-    static constexpr int kStageOff = (kInvLOff + 2 * kBlockM * 4 + 1023) & ~1023;   // one 128 x D bf16 O tile
+    static constexpr int kClockOff = kInvLOff + 2 * kBlockM * 4;                      // int64[2]: start clock, timer
+    static constexpr int kStageOff = (kClockOff + 16 + 1023) & ~1023;   // one 128 x D bf16 O tile
     static constexpr int kBytes = kStageOff + kTileBytes;
     static constexpr int kSmemBytes = kBytes + 1024;           // slack for 1024-byte alignment
     static constexpr uint32_t kTmemS = 0;
@@ -110,7 +111,33 @@ struct Params {
     int num_units;       // bh * num_qblocks
     float scale_log2;    // scale * log2(e)
     int skip_one_arrival;  // test hook: CTA 0 never loads its first Q tile (one wait runs out)
+    unsigned long long* clock;  // null, or [0] SM cycles, [1] timer ns, [2] CTAs: summed over CTAs
 };
+
+// Global timer in nanoseconds (%globaltimer).
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Clock record: each CTA adds the SM cycles and global-timer nanoseconds it
+// ran, and one to the CTA count (the start values wait in shared memory).
+__device__ __forceinline__ void clock_start(const Params& p, uint8_t* slot) {
+    if (threadIdx.x == 0 && p.clock) {
+        reinterpret_cast<long long*>(slot)[0] = clock64();
+        reinterpret_cast<unsigned long long*>(slot)[1] = globaltimer();
+    }
+}
+__device__ __forceinline__ void clock_end(const Params& p, const uint8_t* slot) {
+    if (threadIdx.x == 0 && p.clock) {
+        const long long c = clock64() - reinterpret_cast<const long long*>(slot)[0];
+        const unsigned long long t = globaltimer() - reinterpret_cast<const unsigned long long*>(slot)[1];
+        atomicAdd(p.clock, static_cast<unsigned long long>(c));
+        atomicAdd(p.clock + 1, t);
+        atomicAdd(p.clock + 2, 1ull);
+    }
+}
 
 struct Sync {
     volatile int* abort;
@@ -211,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw);
+    clock_start(p, smem + L::kClockOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -826,6 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
+    clock_end(p, smem + L::kClockOff);
 }
 
 }  // namespace tc
