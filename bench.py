@@ -335,8 +335,7 @@ def run_ours(a, w: W.Workload):
             "frac": tflops_rank / peak, "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
             "frac_of_sustained": tflops_rank / peak_sus,
             "traffic": traffic_from_profile(w), "algorithmic_bytes": alg_bytes,
-            "kernel": f"fa_fwd_bf16_kernel<{w.d},{str(w.causal).lower()}>" if w.dtype == torch.bfloat16
-            else f"fa_fwd_f32_kernel<{w.d},{str(w.causal).lower()}>",
+            "kernel": fa.forward_kernel_name(w.B, w.H, w.N, w.d, w.causal, w.dtype),
             "hbm_gbs_at_algorithmic_bytes": alg_bytes / (ms * 1e-3) / 1e9}
         line["clocks"] = clocks.summary()
         add_in_kernel_clock(line, in_kernel, a.steps)
@@ -863,7 +862,7 @@ def run_ring(a, w: W.Workload):
                        "flop_per_step": flops},
             "roofline": {"bound": "tensor", "achieved": tf / world, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / world / peak, "peak_kind": f"{peak_kind} dense bf16 burst (cuBLAS)",
-                         "traffic": None, "kernel": "fa_fwd_bf16_kernel per chunk pair + fa_merge_kernel"},
+                         "traffic": None, "kernel": "bf16 forward kernel (chosen by size) per chunk pair + fa_merge_kernel"},
             "clocks": clocks.summary(),
             "gpu_launches": a.steps * ring_launches_per_rank(chunks, w.causal) * (1 if world > 1 else chunks)}
     add_cycles(line, ms)

@@ -251,3 +251,19 @@ def test_fp8_output_is_twice_the_input_bytes(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_fp8_needs_a_gpu(lib):
     assert call_fp8(lib) == fa.FA_ERR_CUDA
+
+
+def test_force_forward_kernel_hook(lib):
+    # the test hook only records the choice: no CUDA call, so it runs here
+    for bad in (3, -1, 99):
+        assert lib.fa_test_force_forward_kernel(bad) == fa.FA_ERR_INVALID_ARGUMENT
+        assert "0, 1 or 2" in lib.fa_last_error().decode()
+    for ok in (1, 2, 0):
+        assert lib.fa_test_force_forward_kernel(ok) == fa.FA_OK
+
+
+def test_clock_record_arguments(lib):
+    assert lib.fa_clock_record(None, 0, None) == fa.FA_ERR_INVALID_ARGUMENT
+    if not torch.cuda.is_available():
+        out = (ctypes.c_int64 * 3)()
+        assert lib.fa_clock_record(None, 1, out) == fa.FA_ERR_CUDA

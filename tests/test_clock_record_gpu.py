@@ -13,20 +13,22 @@ from tiled_exact_attention_fa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _grid(B, H, N):
-    units = B * H * ((N + 255) // 256)
+def _grid(B, H, N, rows):
+    units = B * H * ((N + rows - 1) // rows)
     return min(units, torch.cuda.get_device_properties(0).multi_processor_count)
 
 
-def test_clock_record_counts_every_cta():
+@pytest.mark.parametrize("which,rows", [(1, 256), (2, 128)], ids=["two_tile", "one_tile"])
+def test_clock_record_counts_every_cta(which, rows, force_kernel):
     fa_build.build()
-    B, H, N, d = 1, 4, 1000, 128  # 16 units: a grid smaller than the SM count
+    force_kernel(which)
+    B, H, N, d = 1, 4, 1000, 128  # a grid smaller than the SM count
     q, k, v = (x.cuda() for x in W.random_qkv(B, H, N, d, torch.bfloat16, seed=5))
     fa.clock_record(reset=True)
     for _ in range(3):
         fa.forward(q, k, v, causal=True)
     rec = fa.clock_record(reset=True)
-    assert rec["ctas"] == 3 * _grid(B, H, N)
+    assert rec["ctas"] == 3 * _grid(B, H, N, rows)
     assert rec["cycles"] > 0 and rec["ns"] > 0
     assert 200.0 < rec["sm_mhz"] < 2500.0
     assert fa.clock_record(reset=False)["ctas"] == 0  # cleared by the reset
@@ -34,12 +36,12 @@ def test_clock_record_counts_every_cta():
 
 def test_clock_record_full_grid_and_fp8_and_noalloc():
     fa_build.build()
-    B, H, N, d = 2, 32, 2048, 128  # 512 units: one CTA per SM
+    B, H, N, d = 2, 32, 2048, 128  # 512 two-tile units: one CTA per SM
     q, k, v = (x.cuda() for x in W.random_qkv(B, H, N, d, torch.bfloat16, seed=6))
     fa.clock_record(reset=True)
     fa.forward(q, k, v, causal=False)
     rec = fa.clock_record(reset=True)
-    assert rec["ctas"] == _grid(B, H, N)
+    assert rec["ctas"] == _grid(B, H, N, 256)
     # every CTA runs from the first unit to the queue's end: its cycles are
     # close to the launch's, so the per-CTA figure and the clock agree
     assert rec["cycles_per_cta"] > 0
@@ -47,7 +49,7 @@ def test_clock_record_full_grid_and_fp8_and_noalloc():
 
     q8, k8, v8 = (x.to(torch.float8_e4m3fn) for x in (q, k, v))
     fa.forward_fp8(q8, k8, v8, causal=True)
-    assert fa.clock_record(reset=True)["ctas"] == _grid(B, H, N)
+    assert fa.clock_record(reset=True)["ctas"] == _grid(B, H, N, 256)
 
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)

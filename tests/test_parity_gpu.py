@@ -27,6 +27,14 @@ def _built():
     fa.library()
 
 
+@pytest.fixture(autouse=True, params=[1, 2], ids=["two_tile", "one_tile"])
+def forward_kernel(request, force_kernel):
+    """Every test runs on each bf16 forward kernel (256-row units with two
+    query tiles per CTA, and 128-row units); the f32 path ignores the choice."""
+    force_kernel(request.param)
+    return request.param
+
+
 def run_guarded(q, k, v, scale, causal, stream=None):
     """fa_fwd through the C ABI into NaN-filled, guard-banded outputs on the GPU."""
     B, H, N, d = q.shape
@@ -121,6 +129,19 @@ def test_deterministic_and_stream():
         o2, l2 = run_guarded(q, k, v, 0.1, True, stream=s)
     s.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 3, 640, 64, True), (2, 4, 1000, 128, False),
+                                             (1, 2, 1025, 128, True), (3, 5, 129, 64, False)])
+def test_both_kernels_bit_identical(B, H, N, d, causal, force_kernel):
+    # same arithmetic in the same order (S, the lazily moved max, both row
+    # sums, P V per block, 1/l): the two bf16 kernels agree bit for bit
+    q, k, v = (x.cuda() for x in W.random_qkv(B, H, N, d, torch.bfloat16, seed=7 * N + d))
+    outs = []
+    for which in (1, 2):
+        force_kernel(which)
+        outs.append(run_guarded(q, k, v, 1 / math.sqrt(d), causal))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
 def test_causal_row0_is_exact():

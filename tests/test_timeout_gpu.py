@@ -16,9 +16,11 @@ from tiled_exact_attention_fa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_runs_out_and_is_reported():
+@pytest.mark.parametrize("which", [1, 2], ids=["two_tile", "one_tile"])
+def test_bounded_wait_runs_out_and_is_reported(which, force_kernel):
     fa_build.build()
     lib = fa.library()
+    force_kernel(which)
     q, k, v = (x.cuda() for x in W.random_qkv(1, 2, 512, 128, torch.bfloat16, seed=71))
     fa.check_device_status()  # start clean
     assert lib.fa_test_skip_one_arrival() == fa.FA_OK

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "fa_version": (ctypes.c_int, []),
     # include/fa_testing.h
     "fa_test_skip_one_arrival": (ctypes.c_int, []),
+    "fa_test_force_forward_kernel": (ctypes.c_int, [ctypes.c_int]),
 }
 
 _lib = None
@@ -336,6 +337,22 @@ def check_device_status(stream: torch.cuda.Stream | None = None) -> None:
     """Synchronise and raise FaError(FA_ERR_DEVICE_TIMEOUT) if a kernel gave up on a wait."""
     s = (stream or torch.cuda.current_stream()).cuda_stream
     _check(int(library().fa_check_device_status(s)))
+
+
+def forward_kernel_name(B: int, H: int, N: int, d: int, causal: bool, dtype=torch.bfloat16,
+                        sm_count: int | None = None) -> str:
+    """The kernel fa_fwd launches for this problem, by the library's own rule:
+    bf16 takes the one-tile kernel (128-row units) when B * H * ceil(N / 128)
+    is at most the SM count, else the two-tile kernel (256-row units); fp32
+    takes the CUDA-core kernel.  For labels (bench lines, profiles)."""
+    c = str(bool(causal)).lower()
+    if dtype != torch.bfloat16:
+        return f"fa_fwd_f32_kernel<{d},{c}>"
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    if B * H * ((N + 127) // 128) <= sm_count:
+        return f"fa_fwd_bf16_tile_kernel<{d},{c}>"
+    return f"fa_fwd_bf16_kernel<{d},{c}>"
 
 
 def clock_record(reset: bool = True, stream: torch.cuda.Stream | None = None) -> dict:

@@ -25,6 +25,7 @@
 #include "fa_fwd_fp8_tc.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
+#include "fa_fwd_tc1.cuh"
 
 namespace {
 
@@ -64,6 +65,7 @@ struct DeviceState {
     int sm_count = 0;
     int cc_major = 0;
     bool smem_raised[4] = {false, false, false, false};
+    bool tile_smem_raised[4] = {false, false, false, false};
     bool decode_smem_raised[8] = {false, false, false, false, false, false, false, false};
     bool bwd_smem_raised[8] = {false, false, false, false, false, false, false, false};
     bool fp8_smem_raised[2] = {false, false};
@@ -73,6 +75,8 @@ struct DeviceState {
 constexpr int kMaxDevices = 64;
 // set by fa_test_skip_one_arrival; consumed by the next bf16 launch of fa_fwd
 std::atomic<int> g_skip_one_arrival{0};
+// set by fa_test_force_forward_kernel: 0 by problem size, 1 two-tile, 2 one-tile
+std::atomic<int> g_force_forward_kernel{0};
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -167,6 +171,45 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     return FA_OK;
 }
 
+// The one-tile kernel (fa_fwd_tc1.cuh): 128-row units, one CTA per unit up
+// to the SM count.
+template <int D, bool kCausal>
+int launch_bf16_tile(DeviceState* st, int slot, const void* q, const void* k, const void* v, void* o, float* lse,
+                     int64_t bh, int64_t n, float scale, cudaStream_t stream) {
+    using L = fa::tc1::Layout<D>;
+    auto kernel = fa::tc1::fa_fwd_bf16_tile_kernel<D, kCausal>;
+    if (!st->tile_smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->tile_smem_raised[slot] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+
+    fa::tc::Params p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.status = st->status;
+    p.sched = st->queues + 2 * (st->next_queue.fetch_add(1, std::memory_order_relaxed) % kQueues);
+    p.bh = static_cast<int>(bh);
+    p.n = static_cast<int>(n);
+    p.num_qblocks = static_cast<int>((n + fa::tc::kBlockM - 1) / fa::tc::kBlockM);  // 128-row units
+    p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
+    p.num_units = p.bh * p.num_qblocks;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.skip_one_arrival = g_skip_one_arrival.exchange(0);
+    p.clock = st->clock;
+    const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
+    kernel<<<grid, fa::tc1::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the one-tile bf16 attention kernel");
+    return FA_OK;
+}
+
 template <int D, bool kCausal>
 int launch_f32(const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh, int64_t n,
                float scale, cudaStream_t stream) {
@@ -234,6 +277,15 @@ int dispatch(DeviceState* st, const void* q, const void* k, const void* v, void*
     if (dtype == FA_DTYPE_BF16) {
         if (st->cc_major != 10)
             return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
+        // one CTA per 128-row tile when that fits on the GPU at once
+        const int force = g_force_forward_kernel.load();
+        const int64_t tiles = bh * ((N + fa::tc::kBlockM - 1) / fa::tc::kBlockM);
+        if (force == 2 || (force == 0 && tiles <= st->sm_count)) {
+            if (d == 128) return c ? launch_bf16_tile<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
+                                   : launch_bf16_tile<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
+            return c ? launch_bf16_tile<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
+                     : launch_bf16_tile<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
+        }
         if (d == 128) return c ? launch_bf16<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
                                : launch_bf16<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
         return c ? launch_bf16<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
@@ -251,6 +303,13 @@ extern "C" {
 
 int fa_test_skip_one_arrival(void) {
     g_skip_one_arrival.store(1);
+    return FA_OK;
+}
+
+int fa_test_force_forward_kernel(int which) {
+    g_last_error.clear();
+    if (which < 0 || which > 2) return fail(FA_ERR_INVALID_ARGUMENT, "which must be 0, 1 or 2");
+    g_force_forward_kernel.store(which);
     return FA_OK;
 }
 
