@@ -70,6 +70,7 @@ def code_digest(files=None) -> str:
 # the sources each kernel is compiled from (for records tied to one kernel)
 KERNEL_SOURCES = {
     "forward": ["fa_fwd_tc.cuh", "sm100_ptx.cuh"],
+    "forward_tile": ["fa_fwd_tc1.cuh", "fa_fwd_tc.cuh", "sm100_ptx.cuh"],
     "decode": ["fa_decode.cuh", "sm100_ptx.cuh"],
     "decode_mma": ["fa_decode_mma.cuh", "fa_decode.cuh", "sm100_ptx.cuh"],
     "forward_fp8": ["fa_fwd_fp8_tc.cuh", "fa_fwd_tc.cuh", "sm100_ptx.cuh"],
