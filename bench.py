@@ -102,8 +102,12 @@ def traffic_from_profile(w, kind: str | None = None):
         d = json.load(f)
     if kind is None and isinstance(w, W.DecodeWorkload):
         kind = "decode_mma" if w.dtype == torch.bfloat16 else "decode"
+    elif kind is None and w.dtype == torch.float8_e4m3fn:
+        kind = "forward_fp8"
     elif kind is None:
-        kind = "forward_fp8" if w.dtype == torch.float8_e4m3fn else "forward"
+        import tiled_exact_attention_fa_b200 as fa_pkg
+        tile = "tile" in fa_pkg.forward_kernel_name(w.B, w.H, w.N, w.d, w.causal, w.dtype)
+        kind = "forward_tile" if tile else "forward"
     if d.get("kernel_digest") != kernel_digest(kind):
         return None
     return d.get("dram_bytes_per_launch")

@@ -267,3 +267,13 @@ def test_clock_record_arguments(lib):
     if not torch.cuda.is_available():
         out = (ctypes.c_int64 * 3)()
         assert lib.fa_clock_record(None, 1, out) == fa.FA_ERR_CUDA
+
+
+def test_forward_kernel_name_follows_the_size_rule():
+    # one-tile kernel while B * H * ceil(N / 128) <= SM count
+    name = fa.forward_kernel_name
+    assert name(1, 8, 2048, 64, False, sm_count=148) == "fa_fwd_bf16_tile_kernel<64,false>"   # 128 tiles
+    assert name(1, 1, 148 * 128, 128, True, sm_count=148) == "fa_fwd_bf16_tile_kernel<128,true>"
+    assert name(1, 1, 148 * 128 + 1, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
+    assert name(2, 32, 8192, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
+    assert name(1, 1, 256, 64, False, torch.float32, sm_count=148) == "fa_fwd_f32_kernel<64,false>"
