@@ -251,3 +251,32 @@ def test_score_jump_inside_a_block(d, jump_at):
     v = torch.randn(1, 2, N, d, generator=g)
     q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
     check_against_oracle(q, k, v, 1.0 / 8.0, False, strict_raw=False)
+
+
+def test_dependent_launches_keep_stream_order():
+    # The forward kernels start while the previous kernel of the stream is
+    # still running and wait for it before touching memory.  A chain where
+    # each forward reads the previous forward's O as its Q, with torch
+    # kernels writing and reading the buffers in between, must give exactly
+    # the results of the same calls with a synchronisation after each one.
+    q, k, v = (x.cuda() for x in W.random_qkv(1, 4, 700, 128, torch.bfloat16, seed=97))
+    scale = 1 / math.sqrt(128)
+
+    def chain(sync):
+        outs, cur = [], q
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], device="cuda")
+        for i in range(12):
+            o.fill_(float("nan"))                       # a torch kernel writes O first
+            fa.forward_into(cur, k, v, o, lse, scale=scale, causal=i % 2 == 1)
+            if sync:
+                torch.cuda.synchronize()
+            outs.append((o.clone(), lse.clone()))       # and one reads it right after
+            cur = (o * 4.0).to(torch.bfloat16)          # the next Q comes from this O
+        torch.cuda.synchronize()
+        return outs
+
+    for (o1, l1), (o2, l2) in zip(chain(False), chain(True)):
+        assert not torch.isnan(o1).any()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    fa.check_device_status()

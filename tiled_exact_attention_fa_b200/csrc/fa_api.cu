@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
+#include <utility>
 #include <string>
 
 #include "fa.h"
@@ -113,6 +114,26 @@ int device_state(DeviceState** out) {
     return FA_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// (shared memory, barriers, tensor memory) while the previous kernel of the
+// stream finishes; the kernel waits for it (griddepcontrol.wait) before it
+// touches global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(Params...), int grid, int threads, int smem, cudaStream_t stream,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return x < y + nb && y < x + na;
@@ -165,8 +186,8 @@ int launch_bf16(DeviceState* st, int slot, const void* q, const void* k, const v
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     p.clock = st->clock;
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
-    kernel<<<grid, fa::tc::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_overlapped(kernel, grid, fa::tc::kThreads, L::kSmemBytes, stream, tq, tk, tv, to, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the bf16 attention kernel");
     return FA_OK;
 }
@@ -204,8 +225,8 @@ int launch_bf16_tile(DeviceState* st, int slot, const void* q, const void* k, co
     p.skip_one_arrival = g_skip_one_arrival.exchange(0);
     p.clock = st->clock;
     const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
-    kernel<<<grid, fa::tc1::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_overlapped(kernel, grid, fa::tc1::kThreads, L::kSmemBytes, stream, tq, tk, tv, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the one-tile bf16 attention kernel");
     return FA_OK;
 }
@@ -1084,8 +1105,8 @@ int launch_e4m3(DeviceState* st, const void* q, const void* k, const void* v, vo
     p.base.clock = st->clock;
     p.o_scale = o_scale;
     const int grid = p.base.num_units < st->sm_count ? p.base.num_units : st->sm_count;
-    kernel<<<grid, fa::tc8::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_overlapped(kernel, grid, fa::tc8::kThreads, L::kSmemBytes, stream, tq, tk, tv, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch of the E4M3 attention kernel");
     return FA_OK;
 }

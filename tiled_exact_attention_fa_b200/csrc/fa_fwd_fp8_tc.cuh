@@ -214,7 +214,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw);
-    tc::clock_start(p, smem + L::kClockOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -278,9 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
+    tc::grid_dependency_wait();
     const uint32_t tmem = *tmem_base_ptr;
 
     if (warp == kLoadWarp) {
+        tc::clock_start(p, smem + L::kClockOff, lane == 0);
         // ------------------------------------------------------------ producer
         const bool leader = ptx::elect_one();
         const uint64_t keep = ptx::policy_evict_last();   // K/V: re-read by the head's other units
@@ -301,7 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_arrive(sched_full(rs));
             }
             u = __shfl_sync(0xffffffffu, u, __ffs(__ballot_sync(0xffffffffu, leader)) - 1);
-            if (u < 0) break;
+            if (u < 0) {
+                tc::launch_dependents();
+                break;
+            }
 
             const tc::Unit w = tc::decode_unit(u, p, kCausal);
             const int n1 = tc::num_kv_blocks(p, w.qb, 1, kCausal);

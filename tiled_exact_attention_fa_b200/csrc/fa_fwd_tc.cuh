@@ -121,10 +121,19 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// Programmatic dependent launch (the kernels are launched with programmatic
+// stream serialization): a CTA may start while the previous kernel of the
+// stream is still running.  It sets up shared memory, barriers and tensor
+// memory, then waits for that kernel to complete (and its writes to be
+// visible) before it touches global memory; once its producer finds the work
+// queue empty it lets the next kernel's CTAs start on SMs that free up.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // Clock record: each CTA adds the SM cycles and global-timer nanoseconds it
 // ran, and one to the CTA count (the start values wait in shared memory).
-__device__ __forceinline__ void clock_start(const Params& p, uint8_t* slot) {
-    if (threadIdx.x == 0 && p.clock) {
+__device__ __forceinline__ void clock_start(const Params& p, uint8_t* slot, bool me) {
+    if (me && p.clock) {
         reinterpret_cast<long long*>(slot)[0] = clock64();
         reinterpret_cast<unsigned long long*>(slot)[1] = globaltimer();
     }
@@ -238,7 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw);
-    clock_start(p, smem + L::kClockOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -305,9 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
+    grid_dependency_wait();
     const uint32_t tmem = *tmem_base_ptr;
 
     if (warp == kLoadWarp) {
+        clock_start(p, smem + L::kClockOff, lane == 0);
         // ------------------------------------------------------------ producer
         // The whole warp runs the loop (warp-uniform addresses and waits);
         // one elected lane issues the copies.
@@ -331,7 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_arrive(sched_full(rs));
             }
             u = __shfl_sync(0xffffffffu, u, __ffs(__ballot_sync(0xffffffffu, leader)) - 1);
-            if (u < 0) break;
+            if (u < 0) {
+                launch_dependents();
+                break;
+            }
 
             const Unit w = decode_unit(u, p, kCausal);
             const int n1 = num_kv_blocks(p, w.qb, 1, kCausal);
