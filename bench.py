@@ -173,6 +173,50 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(loaded)}
 
 
+def pcie_bandwidth(dev, in_bytes: int, out_bytes: int) -> dict:
+    """Host<->device copy rates with pinned buffers (best of 4, CUDA events):
+    each direction alone, and the time to move one step's bytes in and out
+    at the same time on two streams -- the copy bound of an end-to-end step."""
+    h_in = torch.empty(in_bytes, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+    h_out = torch.empty(out_bytes, dtype=torch.uint8, pin_memory=True)
+    d_out = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev)
+    s2 = torch.cuda.Stream(dev)
+
+    def best_ms(body):
+        best = None
+        for _ in range(4):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record(s)
+            body()
+            b.record(s)
+            torch.cuda.synchronize(dev)
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    def both():
+        s2.wait_stream(s)
+        d_in.copy_(h_in, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h_out.copy_(d_out, non_blocking=True)
+        s.wait_stream(s2)
+
+    out = {"h2d_gbs": in_bytes / (best_ms(lambda: d_in.copy_(h_in, non_blocking=True)) * 1e-3) / 1e9,
+           "d2h_gbs": out_bytes / (best_ms(lambda: h_out.copy_(d_out, non_blocking=True)) * 1e-3) / 1e9,
+           "both_directions_ms": best_ms(both)}
+    return out
+
+
+def add_pcie_roofline(e2e: dict) -> None:
+    """The step's copy time (both directions at once, measured) beside the
+    step's time: the fraction of the end-to-end roofline reached."""
+    bw = e2e["pcie"]
+    bw["frac_of_copy_bound"] = bw["both_directions_ms"] / e2e["ms_per_step"]
+
+
 def add_in_kernel_clock(line: dict, rec: dict, steps: int) -> None:
     """The SM clock the forward kernels themselves saw over the timed steps
     (each CTA's clock64 cycles over its global-timer nanoseconds, summed over
@@ -363,7 +407,9 @@ def run_ours(a, w: W.Workload):
         line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                        "h2d_bytes_per_step": in_bytes,
                        "d2h_bytes_per_step": o.numel() * o.element_size() + lse.numel() * 4,
-                       "api": "tiled_exact_attention_fa_b200.forward(host pinned tensors, out=host pinned) -> fa_fwd_host (C ABI; chunked, pipelined copies)"}
+                       "api": "tiled_exact_attention_fa_b200.forward(host pinned tensors, out=host pinned) -> fa_fwd_host (C ABI; chunked, pipelined copies)",
+                       "pcie": pcie_bandwidth(dev, in_bytes, o.numel() * o.element_size() + lse.numel() * 4)}
+        add_pcie_roofline(line["e2e"])
         if "value" not in line:
             line["value"] = line["e2e"]["value"]
 
