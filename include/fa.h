@@ -169,6 +169,17 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                float descale_q, float descale_k, float descale_v, int causal, void* stream);
 
 /*
+ * fa_fwd_fp8_host -- fa_fwd_fp8 on buffers in host memory: the same
+ * operation, arguments, layouts, results and errors as fa_fwd_fp8, with q, k,
+ * v, o and lse allowed to be host pointers, and the same chunked pipeline of
+ * copy-in, kernel and copy-out (and the same staging buffers and ordering on
+ * `stream`) as fa_fwd_host.  No alignment is required.
+ */
+int fa_fwd_fp8_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+                    float descale_q, float descale_k, float descale_v, int causal, void* stream);
+
+/*
  * fa_fwd_host -- fa_fwd on buffers in host memory: the same operation,
  * arguments, layouts, results and errors, but q, k, v, o and lse may be host
  * pointers (page-locked memory, e.g. from cudaHostAlloc, for the copies to

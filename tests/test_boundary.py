@@ -277,3 +277,24 @@ def test_forward_kernel_name_follows_the_size_rule():
     assert name(1, 1, 148 * 128 + 1, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
     assert name(2, 32, 8192, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
     assert name(1, 1, 256, 64, False, torch.float32, sm_count=148) == "fa_fwd_f32_kernel<64,false>"
+
+
+def call_fp8_host(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,
+                  scale=0.1, dq=1.0, dk=1.0, dv=1.0, causal=0):
+    return lib.fa_fwd_fp8_host(q, k, v, o, lse, B, H, N, d, scale, dq, dk, dv, causal, None)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(N=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(dq=float("inf")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(o=A + 2 * NB - 64), fa.FA_ERR_INVALID_ARGUMENT),   # bf16 o reaches v
+    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_host_rejected_before_cuda(lib, kwargs, code):
+    assert call_fp8_host(lib, **kwargs) == code
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_fp8_host_needs_no_alignment_but_a_gpu(lib):
+    assert call_fp8_host(lib, q=A + 3) == fa.FA_ERR_CUDA

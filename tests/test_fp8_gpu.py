@@ -140,3 +140,16 @@ def test_workloads(w):
     q, k, v = W.make_inputs(w)
     stats, _, _ = check_fp8(q, k, v, w.scale, w.causal, rows=W.sample_rows(w))
     print(w.name, stats)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_host_buffers_match_device_path(causal):
+    # fa_fwd_fp8_host (pinned host tensors, chunks of heads through the
+    # copy/kernel/copy pipeline) gives the device path's result bit for bit;
+    # 2 x 9 heads make several chunks, N = 700 a ragged last tile
+    q, k, v = e4m3_qkv(2, 9, 700, seed=71)
+    o_d, l_d = fa.forward_fp8(q.cuda(), k.cuda(), v.cuda(), descale_v=0.5, causal=causal)
+    o_h, l_h = fa.forward_fp8(q.pin_memory(), k.pin_memory(), v.pin_memory(), descale_v=0.5, causal=causal)
+    fa.check_device_status()
+    assert not o_h.is_cuda
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())

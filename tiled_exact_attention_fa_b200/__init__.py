@@ -38,6 +38,8 @@ _SIGNATURES = {
                    [ctypes.c_float] * 4 + [ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
                     [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "fa_fwd_fp8_host": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 +
+                        [ctypes.c_float] * 4 + [ctypes.c_int, ctypes.c_void_p]),
     "fa_decode": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 5 +
                   [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fa_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 5),
@@ -135,9 +137,12 @@ def forward_fp8_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch
                      lse: torch.Tensor, *, descale_q: float = 1.0, descale_k: float = 1.0,
                      descale_v: float = 1.0, scale: float | None = None, causal: bool = False,
                      stream: torch.cuda.Stream | None = None) -> None:
-    """fa_fwd_fp8: q, k, v torch.float8_e4m3fn [B, H, N, 128] CUDA tensors,
-    each standing for its values times its descale factor; o bf16 [B, H, N,
-    128] and lse fp32 [B, H, N], caller-provided."""
+    """fa_fwd_fp8: q, k, v torch.float8_e4m3fn [B, H, N, 128] tensors, each
+    standing for its values times its descale factor; o bf16 [B, H, N, 128]
+    and lse fp32 [B, H, N], caller-provided.  All CUDA tensors (asynchronous
+    on `stream`), or all host tensors (fa_fwd_fp8_host: chunks of heads copied
+    in, computed and copied out in a pipeline; valid once `stream` is
+    synchronised)."""
     if not (q.dtype == k.dtype == v.dtype == torch.float8_e4m3fn):
         raise TypeError("q, k, v must be torch.float8_e4m3fn")
     if o.dtype != torch.bfloat16 or lse.dtype != torch.float32:
@@ -146,27 +151,43 @@ def forward_fp8_into(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch
         raise ValueError("q, k, v, o must share one [B, H, N, d] shape")
     if lse.shape != q.shape[:3]:
         raise ValueError("lse must be [B, H, N]")
+    on_device = [t.is_cuda for t in (q, k, v, o, lse)]
+    if any(on_device) and not all(on_device):
+        raise ValueError("forward_fp8_into takes all CUDA tensors or all host tensors")
     for t in (q, k, v, o, lse):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("forward_fp8_into needs contiguous CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("forward_fp8_into needs contiguous tensors")
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
-    with torch.cuda.device(q.device):
-        _check(int(library().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                        B, H, N, d, float(scale), float(descale_q), float(descale_k),
-                                        float(descale_v), int(causal), s)))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, float(scale),
+            float(descale_q), float(descale_k), float(descale_v), int(causal))
+    if all(on_device):
+        s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+        with torch.cuda.device(q.device):
+            _check(int(library().fa_fwd_fp8(*args, s)))
+    else:
+        # host tensors (pinned for asynchronous copies): fa_fwd_fp8_host on the
+        # current device; o and lse are valid once `stream` is synchronised
+        s = (stream or torch.cuda.current_stream()).cuda_stream
+        _check(int(library().fa_fwd_fp8_host(*args, s)))
 
 
 def forward_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, descale_q: float = 1.0,
                 descale_k: float = 1.0, descale_v: float = 1.0, scale: float | None = None,
                 causal: bool = False, stream: torch.cuda.Stream | None = None):
-    """(o bf16, lse fp32) of the attention over E4M3 inputs (see forward_fp8_into)."""
-    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    """(o bf16, lse fp32) of the attention over E4M3 inputs (see forward_fp8_into).
+    Host inputs give pinned host outputs that are complete when the call returns."""
+    if q.is_cuda:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
     forward_fp8_into(q, k, v, o, lse, descale_q=descale_q, descale_k=descale_k, descale_v=descale_v,
                      scale=scale, causal=causal, stream=stream)
+    if not q.is_cuda:
+        (stream or torch.cuda.current_stream()).synchronize()
     return o, lse
 
 

@@ -636,29 +636,26 @@ int pipe_reserve(HostPipe& pp, size_t bytes) {
     return FA_OK;
 }
 
-}  // namespace
-
-extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-                           int64_t N, int64_t d, float scale, int causal, int dtype, void* stream) {
-    g_last_error.clear();
-    Sizes z;
-    int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, dtype, false, &z);
-    if (rc != FA_OK) return rc;
-    DeviceState* st = nullptr;
-    if ((rc = device_state(&st)) != FA_OK) return rc;
+// Copy-in, kernel, copy-out over chunks of heads.  in_head / out_head: bytes
+// of one head of q (k, v alike) and of o; launch(dq, dk, dv, do, dl, heads,
+// stream) runs the kernel on a chunk's device copies.
+template <typename Launch>
+int host_pipeline(const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh, int64_t N,
+                  size_t in_head, size_t out_head, cudaStream_t caller, Launch&& launch) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     HostPipe& pp = g_pipe[dev];
     std::lock_guard<std::mutex> lock(pp.mu);
+    int rc;
     if ((rc = pipe_setup(pp)) != FA_OK) return rc;
 
-    const int64_t ch = (z.bh + kPipeChunks - 1) / kPipeChunks;  // heads per chunk
-    const size_t head_bytes = static_cast<size_t>(N * d * z.elem), head_lse = static_cast<size_t>(N * 4);
-    const size_t t_bytes = round_up(ch * head_bytes, 256), l_bytes = round_up(ch * head_lse, 256);
-    if ((rc = pipe_reserve(pp, 4 * t_bytes + l_bytes)) != FA_OK) return rc;
+    const int64_t ch = (bh + kPipeChunks - 1) / kPipeChunks;  // heads per chunk
+    const size_t head_lse = static_cast<size_t>(N * 4);
+    const size_t t_in = round_up(ch * in_head, 256), t_out = round_up(ch * out_head, 256);
+    const size_t l_bytes = round_up(ch * head_lse, 256);
+    if ((rc = pipe_reserve(pp, 3 * t_in + t_out + l_bytes)) != FA_OK) return rc;
 
-    cudaStream_t caller = static_cast<cudaStream_t>(stream);
     auto ck = [&](cudaError_t err, const char* what) { return err == cudaSuccess ? FA_OK : cuda_fail(err, what); };
     if ((rc = ck(cudaEventRecord(pp.ev_entry, caller), "cudaEventRecord")) != FA_OK) return rc;
     if ((rc = ck(cudaStreamWaitEvent(pp.s_in, pp.ev_entry, 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
@@ -667,17 +664,18 @@ extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o,
     const char* hv = static_cast<const char*>(v);
     char* ho = static_cast<char*>(o);
     char* hl = reinterpret_cast<char*>(lse);
-    const int64_t nchunks = (z.bh + ch - 1) / ch;
+    const int64_t nchunks = (bh + ch - 1) / ch;
     for (int64_t i = 0; i < nchunks; ++i) {
         const int b = static_cast<int>(i % kPipeBuffers);
-        const int64_t h0 = i * ch, hc = (h0 + ch <= z.bh) ? ch : z.bh - h0;
-        const size_t off = static_cast<size_t>(h0) * head_bytes, nb = static_cast<size_t>(hc) * head_bytes;
+        const int64_t h0 = i * ch, hc = (h0 + ch <= bh) ? ch : bh - h0;
+        const size_t off = static_cast<size_t>(h0) * in_head, nb = static_cast<size_t>(hc) * in_head;
+        const size_t ooff = static_cast<size_t>(h0) * out_head, onb = static_cast<size_t>(hc) * out_head;
         const size_t loff = static_cast<size_t>(h0) * head_lse, lnb = static_cast<size_t>(hc) * head_lse;
         char* dq = pp.buf[b];
-        char* dk = dq + t_bytes;
-        char* dv = dk + t_bytes;
-        char* dout = dv + t_bytes;
-        float* dl = reinterpret_cast<float*>(dout + t_bytes);
+        char* dk = dq + t_in;
+        char* dv = dk + t_in;
+        char* dout = dv + t_in;
+        float* dl = reinterpret_cast<float*>(dout + t_out);
         // copy-in once the buffer's previous chunk (of this call or an earlier
         // one) has been copied out; an event never recorded is no wait
         if ((rc = ck(cudaStreamWaitEvent(pp.s_in, pp.ev_free[b], 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
@@ -688,11 +686,11 @@ extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o,
             return rc;
         // the kernel on this chunk's heads
         if ((rc = ck(cudaStreamWaitEvent(pp.s_comp, pp.ev_in[b], 0), "cudaStreamWaitEvent")) != FA_OK) return rc;
-        if ((rc = dispatch(st, dq, dk, dv, dout, dl, hc, N, d, scale, causal != 0, dtype, pp.s_comp)) != FA_OK) return rc;
+        if ((rc = launch(dq, dk, dv, dout, dl, hc, pp.s_comp)) != FA_OK) return rc;
         if ((rc = ck(cudaEventRecord(pp.ev_comp[b], pp.s_comp), "cudaEventRecord")) != FA_OK) return rc;
         // copy-out
         if ((rc = ck(cudaStreamWaitEvent(pp.s_out, pp.ev_comp[b], 0), "cudaStreamWaitEvent")) != FA_OK ||
-            (rc = ck(cudaMemcpyAsync(ho + off, dout, nb, cudaMemcpyDefault, pp.s_out), "cudaMemcpyAsync(o)")) != FA_OK ||
+            (rc = ck(cudaMemcpyAsync(ho + ooff, dout, onb, cudaMemcpyDefault, pp.s_out), "cudaMemcpyAsync(o)")) != FA_OK ||
             (rc = ck(cudaMemcpyAsync(hl + loff, dl, lnb, cudaMemcpyDefault, pp.s_out), "cudaMemcpyAsync(lse)")) != FA_OK ||
             (rc = ck(cudaEventRecord(pp.ev_free[b], pp.s_out), "cudaEventRecord")) != FA_OK)
             return rc;
@@ -700,6 +698,24 @@ extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o,
     // the caller's stream continues once the last copy-out is done
     if ((rc = ck(cudaEventRecord(pp.ev_done, pp.s_out), "cudaEventRecord")) != FA_OK) return rc;
     return ck(cudaStreamWaitEvent(caller, pp.ev_done, 0), "cudaStreamWaitEvent");
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                           int64_t N, int64_t d, float scale, int causal, int dtype, void* stream) {
+    g_last_error.clear();
+    Sizes z;
+    int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, dtype, false, &z);
+    if (rc != FA_OK) return rc;
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    const size_t head_bytes = static_cast<size_t>(N * d * z.elem);
+    return host_pipeline(q, k, v, o, lse, z.bh, N, head_bytes, head_bytes, static_cast<cudaStream_t>(stream),
+                         [&](const void* dq, const void* dk, const void* dv, void* dout, float* dl, int64_t hc,
+                             cudaStream_t s) {
+                             return dispatch(st, dq, dk, dv, dout, dl, hc, N, d, scale, causal != 0, dtype, s);
+                         });
 }
 
 // ---------------------------------------------------------------------------
@@ -1113,10 +1129,12 @@ int launch_e4m3(DeviceState* st, const void* q, const void* k, const void* v, vo
 
 }  // namespace
 
-extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-                          int64_t N, int64_t d, float scale, float descale_q, float descale_k, float descale_v,
-                          int causal, void* stream) {
-    g_last_error.clear();
+namespace {
+
+// Arguments of the E4M3 forward; device_pointers adds the alignment checks.
+int check_fp8_args(const void* q, const void* k, const void* v, const void* o, const float* lse, int64_t B,
+                   int64_t H, int64_t N, int64_t d, float scale, float descale_q, float descale_k, float descale_v,
+                   bool device_pointers, int64_t* bh_out, double* scale_qk_out) {
     if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID_ARGUMENT, "null pointer argument");
     if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H, N and d must be >= 1");
     if (!std::isfinite(scale) || !std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v))
@@ -1133,20 +1151,61 @@ extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
     const size_t in_bytes = static_cast<size_t>(bh * N * d), o_bytes = 2 * in_bytes;
     const size_t lse_bytes = static_cast<size_t>(bh * N * 4);
     auto mis = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
-    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16))
-        return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
-    if (mis(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (device_pointers) {
+        if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16))
+            return fail(FA_ERR_INVALID_ARGUMENT, "q, k, v and o must be 16-byte aligned");
+        if (mis(lse, 4)) return fail(FA_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    }
     if (overlaps(o, o_bytes, q, in_bytes) || overlaps(o, o_bytes, k, in_bytes) || overlaps(o, o_bytes, v, in_bytes) ||
         overlaps(o, o_bytes, lse, lse_bytes))
         return fail(FA_ERR_INVALID_ARGUMENT, "o overlaps another argument");
     if (overlaps(lse, lse_bytes, q, in_bytes) || overlaps(lse, lse_bytes, k, in_bytes) ||
         overlaps(lse, lse_bytes, v, in_bytes))
         return fail(FA_ERR_INVALID_ARGUMENT, "lse overlaps another argument");
-    DeviceState* st = nullptr;
-    int rc = device_state(&st);
-    if (rc != FA_OK) return rc;
-    if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the E4M3 kernel needs an sm_100 (B200-class) GPU");
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    *bh_out = bh;
+    *scale_qk_out = scale_qk;
+    return FA_OK;
+}
+
+int e4m3_launch(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh,
+                int64_t N, double scale_qk, float descale_v, bool causal, cudaStream_t s) {
     return causal ? launch_e4m3<true>(st, q, k, v, o, lse, bh, N, scale_qk, descale_v, s)
                   : launch_e4m3<false>(st, q, k, v, o, lse, bh, N, scale_qk, descale_v, s);
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                          int64_t N, int64_t d, float scale, float descale_q, float descale_k, float descale_v,
+                          int causal, void* stream) {
+    g_last_error.clear();
+    int64_t bh = 0;
+    double scale_qk = 0.0;
+    int rc = check_fp8_args(q, k, v, o, lse, B, H, N, d, scale, descale_q, descale_k, descale_v, true, &bh,
+                            &scale_qk);
+    if (rc != FA_OK) return rc;
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the E4M3 kernel needs an sm_100 (B200-class) GPU");
+    return e4m3_launch(st, q, k, v, o, lse, bh, N, scale_qk, descale_v, causal != 0, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int fa_fwd_fp8_host(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                               int64_t H, int64_t N, int64_t d, float scale, float descale_q, float descale_k,
+                               float descale_v, int causal, void* stream) {
+    g_last_error.clear();
+    int64_t bh = 0;
+    double scale_qk = 0.0;
+    int rc = check_fp8_args(q, k, v, o, lse, B, H, N, d, scale, descale_q, descale_k, descale_v, false, &bh,
+                            &scale_qk);
+    if (rc != FA_OK) return rc;
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != FA_OK) return rc;
+    if (st->cc_major != 10) return fail(FA_ERR_UNSUPPORTED, "the E4M3 kernel needs an sm_100 (B200-class) GPU");
+    const size_t head_in = static_cast<size_t>(N * d);  // one byte per element in, bf16 out
+    return host_pipeline(q, k, v, o, lse, bh, N, head_in, 2 * head_in, static_cast<cudaStream_t>(stream),
+                         [&](const void* dq, const void* dk, const void* dv, void* dout, float* dl, int64_t hc,
+                             cudaStream_t s) {
+                             return e4m3_launch(st, dq, dk, dv, dout, dl, hc, N, scale_qk, descale_v, causal != 0, s);
+                         });
 }
