@@ -78,6 +78,14 @@ typedef enum {
  * enqueued.  A device-side timeout (a bounded wait that expired) is not seen
  * here; call fa_check_device_status after the stream has run.
  * Thread safety: concurrent calls from several host threads are allowed.
+ *
+ * Kernels and launch (no effect on the result): bf16 problems whose 128-row
+ * query tiles all fit on the GPU at once (B * H * ceil(N / 128) <= the SM
+ * count) run a kernel with one tile per CTA, larger ones a kernel with two
+ * tiles per CTA; both give the same bits.  The bf16 kernels are launched with
+ * programmatic stream serialization: their CTAs may start setting up while
+ * the previous kernel on `stream` is still running, and wait for it to
+ * complete before they read or write any memory, so stream order holds.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int64_t B, int64_t H, int64_t N, int64_t d,
