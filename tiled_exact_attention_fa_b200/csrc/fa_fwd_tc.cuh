@@ -37,6 +37,12 @@
 //     it, so no softmax thread issues the 128 row-strided stores of a tile.
 //   * Causal: KV blocks entirely above the diagonal are never loaded or
 //     multiplied; only the diagonal block is masked.
+//   * Launched with programmatic stream serialization: a CTA sets up its
+//     barriers and TMEM while the previous kernel of the stream finishes and
+//     waits for it (griddepcontrol.wait) before touching global memory.
+//
+// Problems whose 128-row tiles all fit on the GPU at once run the one-tile
+// kernel of fa_fwd_tc1.cuh instead (same arithmetic, same results).
 //
 // TMEM columns (512 allocated): S_0/P_0 at 0, S_1/P_1 at 128, O_0 at 256,
 // O_1 at 256 + D.  P_t (bf16 pairs) occupies the first 64 columns of S_t.
