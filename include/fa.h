@@ -79,10 +79,9 @@ typedef enum {
  * here; call fa_check_device_status after the stream has run.
  * Thread safety: concurrent calls from several host threads are allowed.
  *
- * Kernels and launch (no effect on the result): bf16 problems whose 128-row
- * query tiles all fit on the GPU at once (B * H * ceil(N / 128) <= the SM
- * count) run a kernel with one tile per CTA, larger ones a kernel with two
- * tiles per CTA; both give the same bits.  The bf16 kernels are launched with
+ * Kernels and launch (no effect on the result): bf16 problems run a kernel
+ * with one 128-row query tile per CTA or one with two, whichever finishes
+ * sooner for the shape (fa_fwd_kernel_choice); both give the same bits.  The bf16 kernels are launched with
  * programmatic stream serialization: their CTAs may start setting up while
  * the previous kernel on `stream` is still running, and wait for it to
  * complete before they read or write any memory, so stream order holds.
@@ -335,6 +334,32 @@ int fa_check_device_status(void* stream);
  * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (out NULL) or FA_ERR_CUDA.
  */
 int fa_clock_record(void* stream, int reset, int64_t* out);
+
+/* The forward kernels fa_fwd can launch (see fa_fwd_kernel_choice). */
+typedef enum {
+    FA_KERNEL_F32 = 0,            /* fp32, CUDA cores */
+    FA_KERNEL_BF16_TWO_TILE = 1,  /* bf16, two 128-row query tiles per CTA (256-row units) */
+    FA_KERNEL_BF16_ONE_TILE = 2   /* bf16, one 128-row query tile per CTA */
+} fa_kernel_t;
+
+/*
+ * fa_fwd_kernel_choice -- which kernel fa_fwd (and fa_fwd_host per chunk of
+ * heads) launches for a problem, written to *kernel as an fa_kernel_t.  Not
+ * part of the method; the choice never changes the result (the two bf16
+ * kernels give the same bits), only the time.  For bf16 the library
+ * simulates how the work units of each kernel would be spread over the SMs
+ * (both take units from a queue in the same order, each CTA the next one
+ * when it is free; a unit costs its KV blocks times a measured cycle count
+ * per block) and takes the shorter schedule: the one-tile kernel when every
+ * 128-row tile gets its own SM, the two-tile kernel from 8 tiles per SM on.
+ *   sm_count  SMs to plan for; < 1 means the current device's (then a CUDA
+ *             call is made, and FA_ERR_CUDA is possible).
+ * The test hook fa_test_force_forward_kernel overrides the choice in fa_fwd
+ * but not here.  Returns FA_OK, FA_ERR_INVALID_ARGUMENT, FA_ERR_UNSUPPORTED
+ * (d other than 64 or 128) or FA_ERR_CUDA.
+ */
+int fa_fwd_kernel_choice(int64_t B, int64_t H, int64_t N, int64_t d, int causal, int dtype,
+                         int sm_count, int* kernel);
 
 /* fa_status_string -- static, never-NULL description of a status code. */
 const char* fa_status_string(int status);

@@ -270,13 +270,30 @@ def test_clock_record_arguments(lib):
 
 
 def test_forward_kernel_name_follows_the_size_rule():
-    # one-tile kernel while B * H * ceil(N / 128) <= SM count
+    # fa_fwd_kernel_choice with a given SM count makes no CUDA call.  Cases
+    # whose faster kernel was measured on a B200 (148 SMs), both masks:
     name = fa.forward_kernel_name
-    assert name(1, 8, 2048, 64, False, sm_count=148) == "fa_fwd_bf16_tile_kernel<64,false>"   # 128 tiles
-    assert name(1, 1, 148 * 128, 128, True, sm_count=148) == "fa_fwd_bf16_tile_kernel<128,true>"
-    assert name(1, 1, 148 * 128 + 1, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
-    assert name(2, 32, 8192, 128, True, sm_count=148) == "fa_fwd_bf16_kernel<128,true>"
+    tile, two = "fa_fwd_bf16_tile_kernel", "fa_fwd_bf16_kernel"
+    assert name(1, 8, 2048, 64, False, sm_count=148) == tile + "<64,false>"   # 128 tiles: one wave
+    assert name(1, 16, 2048, 128, True, sm_count=148) == tile + "<128,true>"  # 256 tiles, causal: 0.71x
+    assert name(1, 8, 4096, 128, True, sm_count=148) == tile + "<128,true>"   # 0.63x
+    assert name(1, 16, 2048, 128, False, sm_count=148) == two + "<128,false>"  # 256 tiles, no mask: 1.10x
+    assert name(1, 16, 4096, 128, True, sm_count=148) == two + "<128,true>"    # 512 tiles, causal: 1.13x
+    assert name(2, 32, 8192, 128, True, sm_count=148) == two + "<128,true>"    # headline, beyond 8 per SM
     assert name(1, 1, 256, 64, False, torch.float32, sm_count=148) == "fa_fwd_f32_kernel<64,false>"
+    # the choice follows the SM count it is given
+    assert name(1, 16, 2048, 128, False, sm_count=512) == tile + "<128,false>"
+
+
+def test_kernel_choice_arguments(lib):
+    out = ctypes.c_int(-1)
+    assert lib.fa_fwd_kernel_choice(1, 1, 128, 128, 0, fa.FA_DTYPE_BF16, 148, None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert lib.fa_fwd_kernel_choice(0, 1, 128, 128, 0, fa.FA_DTYPE_BF16, 148, ctypes.byref(out)) == \
+        fa.FA_ERR_INVALID_ARGUMENT
+    assert lib.fa_fwd_kernel_choice(1, 1, 128, 80, 0, fa.FA_DTYPE_BF16, 148, ctypes.byref(out)) == \
+        fa.FA_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():  # the current device's SM count needs a GPU
+        assert lib.fa_fwd_kernel_choice(1, 1, 128, 128, 0, fa.FA_DTYPE_BF16, 0, ctypes.byref(out)) == fa.FA_ERR_CUDA
 
 
 def call_fp8_host(lib, q=A, k=A + NB, v=A + 2 * NB, o=A + 3 * NB, lse=A + 4 * NB, B=1, H=1, N=128, d=128,

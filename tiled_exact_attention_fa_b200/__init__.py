@@ -49,6 +49,8 @@ _SIGNATURES = {
     "fa_merge": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "fa_check_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fa_fwd_kernel_choice": (ctypes.c_int, [ctypes.c_int64] * 4 + [ctypes.c_int] * 3 +
+                             [ctypes.POINTER(ctypes.c_int)]),
     "fa_clock_record": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]),
     "fa_noalloc_check_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -362,18 +364,16 @@ def check_device_status(stream: torch.cuda.Stream | None = None) -> None:
 
 def forward_kernel_name(B: int, H: int, N: int, d: int, causal: bool, dtype=torch.bfloat16,
                         sm_count: int | None = None) -> str:
-    """The kernel fa_fwd launches for this problem, by the library's own rule:
-    bf16 takes the one-tile kernel (128-row units) when B * H * ceil(N / 128)
-    is at most the SM count, else the two-tile kernel (256-row units); fp32
-    takes the CUDA-core kernel.  For labels (bench lines, profiles)."""
+    """The kernel fa_fwd launches for this problem (fa_fwd_kernel_choice:
+    bf16 takes whichever of the one-tile and two-tile kernels the library's
+    schedule estimate finds faster; fp32 the CUDA-core kernel), for labels
+    in bench lines and profiles.  sm_count None: the current device's."""
+    out = ctypes.c_int(-1)
+    _check(int(library().fa_fwd_kernel_choice(B, H, N, d, int(causal), _DTYPES[dtype], int(sm_count or 0),
+                                               ctypes.byref(out))))
     c = str(bool(causal)).lower()
-    if dtype != torch.bfloat16:
-        return f"fa_fwd_f32_kernel<{d},{c}>"
-    if sm_count is None:
-        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    if B * H * ((N + 127) // 128) <= sm_count:
-        return f"fa_fwd_bf16_tile_kernel<{d},{c}>"
-    return f"fa_fwd_bf16_kernel<{d},{c}>"
+    return {0: f"fa_fwd_f32_kernel<{d},{c}>", 1: f"fa_fwd_bf16_kernel<{d},{c}>",
+            2: f"fa_fwd_bf16_tile_kernel<{d},{c}>"}[out.value]
 
 
 def clock_record(reset: bool = True, stream: torch.cuda.Stream | None = None) -> dict:

@@ -13,7 +13,12 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <functional>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 #include <utility>
 #include <string>
 
@@ -292,16 +297,77 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     return FA_OK;
 }
 
+// Which bf16 kernel runs a problem.  Both kernels take their work units
+// from a queue in the same order (groups of kHeadGroup heads; under the causal
+// mask each group's heaviest query blocks first) and every CTA takes the next
+// unit when it is free, so a launch lasts as long as the busiest CTA of that
+// list schedule.  A unit costs its KV blocks times the cycles one block takes:
+// ~1886 for the one-tile kernel's 128 rows, ~3245 for the two-tile kernel's
+// 256 rows (clock64 traces of both kernels in steady state).  The one-tile
+// kernel is picked when its schedule is the shorter: always when every tile
+// has its own SM, never beyond 8 tiles per SM (there its doubled K/V reads
+// and per-block cost always lose), by simulating both schedules in between
+// (cached per shape).  Measured on 64 shapes (B, H, N in 1..4, 4..64,
+// 1K..16K, d 64 and 128, both masks) this picks the faster kernel in 62.
+constexpr double kCyclesPerBlockOneTile = 1886.0;
+constexpr double kCyclesPerBlockPairTwoTile = 3245.0;
+
+double list_schedule_cycles(int64_t bh, int64_t n, bool causal, bool one_tile, int sms) {
+    const int64_t nb = (n + fa::tc::kBlockN - 1) / fa::tc::kBlockN;
+    const int64_t rows = one_tile ? fa::tc::kBlockM : fa::tc::kUnitRows;
+    const int64_t nq = (n + rows - 1) / rows;
+    const double c = one_tile ? kCyclesPerBlockOneTile : kCyclesPerBlockPairTwoTile;
+    const int64_t units = bh * nq;
+    const int64_t ctas = units < sms ? units : sms;
+    std::priority_queue<double, std::vector<double>, std::greater<double>> busy;
+    for (int64_t i = 0; i < ctas; ++i) busy.push(0.0);
+    double end = 0.0;
+    for (int64_t g0 = 0; g0 < bh; g0 += fa::tc::kHeadGroup) {
+        const int64_t hg = (bh - g0 < fa::tc::kHeadGroup) ? bh - g0 : fa::tc::kHeadGroup;
+        for (int64_t qi = 0; qi < nq; ++qi) {
+            const int64_t qb = causal ? nq - 1 - qi : qi;
+            int64_t blocks = nb;
+            if (causal) {
+                const int64_t last = one_tile ? qb + 1 : 2 * qb + 2;  // through the diagonal block
+                blocks = last < nb ? last : nb;
+            }
+            for (int64_t h = 0; h < hg; ++h) {
+                const double t = busy.top() + c * static_cast<double>(blocks);
+                busy.pop();
+                busy.push(t);
+                end = t > end ? t : end;
+            }
+        }
+    }
+    return end;
+}
+
+bool one_tile_is_faster(int64_t bh, int64_t n, bool causal, int sms) {
+    const int64_t tiles = bh * ((n + fa::tc::kBlockM - 1) / fa::tc::kBlockM);
+    if (tiles <= sms) return true;
+    if (tiles > 8 * static_cast<int64_t>(sms)) return false;
+    static std::mutex mu;
+    static std::map<std::tuple<int64_t, int64_t, bool, int>, bool> cache;
+    const auto key = std::make_tuple(bh, n, causal, sms);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
+    const bool one = list_schedule_cycles(bh, n, causal, true, sms) < list_schedule_cycles(bh, n, causal, false, sms);
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() < 4096) cache.emplace(key, one);
+    return one;
+}
+
 // Kernel choice and launch on `s` for bh heads of N rows (device pointers).
 int dispatch(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int64_t bh,
              int64_t N, int64_t d, float scale, bool c, int dtype, cudaStream_t s) {
     if (dtype == FA_DTYPE_BF16) {
         if (st->cc_major != 10)
             return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
-        // one CTA per 128-row tile when that fits on the GPU at once
         const int force = g_force_forward_kernel.load();
-        const int64_t tiles = bh * ((N + fa::tc::kBlockM - 1) / fa::tc::kBlockM);
-        if (force == 2 || (force == 0 && tiles <= st->sm_count)) {
+        if (force == 2 || (force == 0 && one_tile_is_faster(bh, N, c, st->sm_count))) {
             if (d == 128) return c ? launch_bf16_tile<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
                                    : launch_bf16_tile<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
             return c ? launch_bf16_tile<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
@@ -324,6 +390,29 @@ extern "C" {
 
 int fa_test_skip_one_arrival(void) {
     g_skip_one_arrival.store(1);
+    return FA_OK;
+}
+
+int fa_fwd_kernel_choice(int64_t B, int64_t H, int64_t N, int64_t d, int causal, int dtype, int sm_count,
+                         int* kernel) {
+    g_last_error.clear();
+    if (!kernel) return fail(FA_ERR_INVALID_ARGUMENT, "kernel is null");
+    if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARGUMENT, "B, H and N must be >= 1");
+    if (dtype != FA_DTYPE_F32 && dtype != FA_DTYPE_BF16) return fail(FA_ERR_INVALID_ARGUMENT, "unknown dtype");
+    if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+    if (B > INT_MAX / H) return fail(FA_ERR_INVALID_ARGUMENT, "B * H too large");
+    if (N > (int64_t{1} << 30)) return fail(FA_ERR_INVALID_ARGUMENT, "N too large (max 2^30)");
+    if (dtype == FA_DTYPE_F32) {
+        *kernel = FA_KERNEL_F32;
+        return FA_OK;
+    }
+    if (sm_count < 1) {
+        DeviceState* st = nullptr;
+        int rc = device_state(&st);
+        if (rc != FA_OK) return rc;
+        sm_count = st->sm_count;
+    }
+    *kernel = one_tile_is_faster(B * H, N, causal != 0, sm_count) ? FA_KERNEL_BF16_ONE_TILE : FA_KERNEL_BF16_TWO_TILE;
     return FA_OK;
 }
 
