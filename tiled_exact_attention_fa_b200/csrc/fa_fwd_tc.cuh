@@ -41,8 +41,8 @@
 //     barriers and TMEM while the previous kernel of the stream finishes and
 //     waits for it (griddepcontrol.wait) before touching global memory.
 //
-// Problems whose 128-row tiles all fit on the GPU at once run the one-tile
-// kernel of fa_fwd_tc1.cuh instead (same arithmetic, same results).
+// Small and medium problems can run the one-tile kernel of fa_fwd_tc1.cuh
+// instead (same arithmetic, same results; the host picks by schedule).
 //
 // TMEM columns (512 allocated): S_0/P_0 at 0, S_1/P_1 at 128, O_0 at 256,
 // O_1 at 256 + D.  P_t (bf16 pairs) occupies the first 64 columns of S_t.

@@ -17,9 +17,10 @@
 //     block's scores ready and only wait for P_{j-1} V before touching O;
 //   * each warp stores its rows of O straight from registers at the end of a
 //     unit (small problems: no staging tile, no TMA store).
-// The host picks this kernel when every 128-row tile of the problem gets its
-// own SM (B * H * ceil(N / 128) <= SM count); above that the two-tile kernel,
-// which reads each K/V block once for 256 rows, is faster.
+// The host picks this kernel when a simulation of both kernels' schedules
+// says it finishes first: small problems (every 128-row tile on its own SM)
+// and medium causal ones, where the two-tile kernel's heaviest 256-row unit
+// would set the launch's length.
 #pragma once
 
 #include <cstdint>
