@@ -280,3 +280,20 @@ def test_dependent_launches_keep_stream_order():
         assert not torch.isnan(o1).any()
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
     fa.check_device_status()
+
+
+def _random_shapes(n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        out.append((int(rng.integers(1, 4)), int(rng.integers(1, 41)), int(rng.integers(1, 701)),
+                    int(rng.choice([64, 128])), bool(rng.integers(0, 2))))
+    return out
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", _random_shapes(16, 2024))
+def test_random_shapes(B, H, N, d, causal):
+    # seeded random shapes (B 1-3, H 1-40, N 1-700, both head dims and masks)
+    # on each kernel, every row against the oracle
+    q, k, v = W.random_qkv(B, H, N, d, torch.bfloat16, seed=B * 100003 + H * 1009 + N * 7 + d)
+    check_against_oracle(q, k, v, 1 / math.sqrt(d), causal)
