@@ -57,22 +57,38 @@ __global__ void __launch_bounds__(kThreads)
     float m = -INFINITY, l = 0.f;
 
     const int last_key = kCausal ? min(p.n, row0 + kRows) : p.n;  // exclusive
-    for (int key0 = 0; key0 < last_key; key0 += kKeys) {
-        __syncthreads();
-        // stage K/V rows [key0, key0 + kKeys) (zeros past the end)
-        for (int x = tid; x < kKeys * D / 4; x += kThreads) {
+    // K/V rows [key0, key0 + kKeys) of the next tile are read into registers
+    // while the current tile is computed (zeros past the end), then staged in
+    // shared memory at the top of the next iteration.
+    constexpr int kLoads = kKeys * D / 4 / kThreads;
+    static_assert(kKeys * D / 4 % kThreads == 0, "whole float4 loads per thread");
+    float4 nk[kLoads], nv[kLoads];
+    auto fetch = [&](int key0) {
+#pragma unroll
+        for (int j = 0; j < kLoads; ++j) {
+            const int x = tid + j * kThreads;
             const int kr = x / (D / 4);
             const int kc = (x % (D / 4)) * 4;
-            float4 kv4 = make_float4(0.f, 0.f, 0.f, 0.f), vv4 = kv4;
+            nk[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            nv[j] = nk[j];
             if (key0 + kr < p.n) {
                 const int64_t off = static_cast<int64_t>(key0 + kr) * D + kc;
-                kv4 = *reinterpret_cast<const float4*>(kh + off);
-                vv4 = *reinterpret_cast<const float4*>(vh + off);
+                nk[j] = *reinterpret_cast<const float4*>(kh + off);
+                nv[j] = *reinterpret_cast<const float4*>(vh + off);
             }
-            *reinterpret_cast<float4*>(&sk[kr][kc]) = kv4;
-            *reinterpret_cast<float4*>(&sv[kr][kc]) = vv4;
+        }
+    };
+    if (last_key > 0) fetch(0);
+    for (int key0 = 0; key0 < last_key; key0 += kKeys) {
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kLoads; ++j) {
+            const int x = tid + j * kThreads;
+            *reinterpret_cast<float4*>(&sk[x / (D / 4)][(x % (D / 4)) * 4]) = nk[j];
+            *reinterpret_cast<float4*>(&sv[x / (D / 4)][(x % (D / 4)) * 4]) = nv[j];
         }
         __syncthreads();
+        if (key0 + kKeys < last_key) fetch(key0 + kKeys);
 
         float s[kKeys];
         float tmax = -INFINITY;
