@@ -6,8 +6,8 @@
 // plain fp32 so that fp32 inputs keep fp32 accuracy (a TF32 tensor-core path
 // would round the inputs to 10 mantissa bits).
 //
-// One CTA of 128 threads owns 32 query rows; four threads share a row, each
-// holding every fourth element of q and of the output accumulator, and a
+// One CTA of 256 threads owns 32 query rows; eight threads share a row, each
+// holding every eighth element of q and of the output accumulator, and a
 // 32-key tile of K and V sits in shared memory.
 #pragma once
 
@@ -18,7 +18,8 @@ namespace simt {
 
 constexpr int kRows = 32;     // query rows per CTA
 constexpr int kKeys = 32;     // keys per shared-memory tile
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
+constexpr int kSplit = kThreads / kRows;  // threads per query row
 
 struct Params {
     const float* q;
@@ -33,13 +34,13 @@ struct Params {
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads)
     fa_fwd_f32_kernel(const Params p) {
-    constexpr int kPer = D / 4;  // elements of a row each thread owns
+    constexpr int kPer = D / kSplit;  // elements of a row each thread owns
     __shared__ __align__(16) float sk[kKeys][D];
     __shared__ __align__(16) float sv[kKeys][D];
 
     const int tid = threadIdx.x;
-    const int r = tid >> 2;     // row within the CTA
-    const int part = tid & 3;   // which fourth of the row
+    const int r = tid / kSplit;     // row within the CTA
+    const int part = tid % kSplit;  // which share of the row
     const int64_t head = blockIdx.y;
     const int row0 = blockIdx.x * kRows;
     const int row = row0 + r;
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(kThreads)
     float q[kPer], acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-        q[i] = valid ? qh[static_cast<int64_t>(row) * D + part + 4 * i] : 0.f;
+        q[i] = valid ? qh[static_cast<int64_t>(row) * D + part + kSplit * i] : 0.f;
         acc[i] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
@@ -96,9 +97,9 @@ __global__ void __launch_bounds__(kThreads)
         for (int c = 0; c < kKeys; ++c) {
             float dot = 0.f;
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) dot = fmaf(q[i], sk[c][part + 4 * i], dot);
-            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            for (int i = 0; i < kPer; ++i) dot = fmaf(q[i], sk[c][part + kSplit * i], dot);
+#pragma unroll
+            for (int w = 1; w < kSplit; w <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, w);
             const int key = key0 + c;
             const bool allowed = key < p.n && (!kCausal || key <= row);
             s[c] = allowed ? dot * p.scale : -INFINITY;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int i = 0; i < kPer; ++i) {
             float a = acc[i] * alpha;
 #pragma unroll
-            for (int c = 0; c < kKeys; ++c) a = fmaf(s[c], sv[c][part + 4 * i], a);
+            for (int c = 0; c < kKeys; ++c) a = fmaf(s[c], sv[c][part + kSplit * i], a);
             acc[i] = a;
         }
         m = m_new;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads)
         const float inv_l = 1.f / l;
         float* orow = p.o + (head * p.n + row) * D;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) orow[part + 4 * i] = acc[i] * inv_l;
+        for (int i = 0; i < kPer; ++i) orow[part + kSplit * i] = acc[i] * inv_l;
         if (part == 0) p.lse[head * p.n + row] = m + logf(l);
     }
 }
