@@ -6,7 +6,7 @@
 // plain fp32 so that fp32 inputs keep fp32 accuracy (a TF32 tensor-core path
 // would round the inputs to 10 mantissa bits).
 //
-// One CTA of 256 threads owns 32 query rows; eight threads share a row, each
+// One CTA of 128 threads owns 16 query rows; eight threads share a row, each
 // holding every eighth element of q and of the output accumulator, and a
 // 32-key tile of K and V sits in shared memory.
 #pragma once
@@ -16,9 +16,9 @@
 namespace fa {
 namespace simt {
 
-constexpr int kRows = 32;     // query rows per CTA
+constexpr int kRows = 16;     // query rows per CTA
 constexpr int kKeys = 32;     // keys per shared-memory tile
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
 constexpr int kSplit = kThreads / kRows;  // threads per query row
 
 struct Params {
