@@ -315,3 +315,28 @@ def test_fp8_host_rejected_before_cuda(lib, kwargs, code):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_fp8_host_needs_no_alignment_but_a_gpu(lib):
     assert call_fp8_host(lib, q=A + 3) == fa.FA_ERR_CUDA
+
+
+def test_c_program_uses_the_boundary(lib, tmp_path):
+    # the headers compile as C99 and a C program links against the library
+    # and calls it (the calls below make no CUDA call)
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_fa.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "fa.h"\n#include "fa_testing.h"\n'
+        "int main(void) {\n"
+        "    int kernel = -1;\n"
+        "    int rc = fa_fwd_kernel_choice(1, 8, 2048, 64, 0, FA_DTYPE_BF16, 148, &kernel);\n"
+        "    int bad = fa_fwd(0, 0, 0, 0, 0, 1, 1, 1, 64, 0.1f, 0, FA_DTYPE_BF16, 0);\n"
+        '    printf("%d %d %d %d %s\\n", fa_version(), rc, kernel, bad, fa_status_string(bad));\n'
+        "    return 0;\n}\n")
+    exe = tmp_path / "use_fa"
+    pkg = os.path.dirname(fa.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-L", pkg, "-lfa_b200", "-Wl,-rpath," + pkg, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[:4] == [str(fa.version()), str(fa.FA_OK), "2", str(fa.FA_ERR_INVALID_ARGUMENT)]
+    assert out[4].startswith("FA_ERR_INVALID_ARGUMENT")
