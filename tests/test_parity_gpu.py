@@ -297,3 +297,17 @@ def test_random_shapes(B, H, N, d, causal):
     # on each kernel, every row against the oracle
     q, k, v = W.random_qkv(B, H, N, d, torch.bfloat16, seed=B * 100003 + H * 1009 + N * 7 + d)
     check_against_oracle(q, k, v, 1 / math.sqrt(d), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_long_sequence_sampled_rows(causal):
+    # N = 2^17 + 3 rows in one head (1024 KV blocks, a ragged last one): row
+    # and key offsets far past any small-size test, checked on sampled rows
+    # (the first and last rows, tile edges, random rows) against the oracle
+    N = (1 << 17) + 3
+    q, k, v = W.random_qkv(1, 1, N, 64, torch.bfloat16, seed=131)
+    g = torch.Generator().manual_seed(5)
+    picks = torch.randperm(N, generator=g)[:200]
+    rows = torch.cat([torch.tensor([0, 1, 127, 128, N // 2, N - 129, N - 2, N - 1]), picks]).unique().sort().values
+    rows = rows.view(1, 1, -1).contiguous()
+    check_against_oracle(q, k, v, 1 / 8.0, causal, rows=rows)
