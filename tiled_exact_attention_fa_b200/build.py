@@ -3,7 +3,7 @@
     python -m tiled_exact_attention_fa_b200.build [--verbose-ptxas]
 
 nvcc cross-compiles without a GPU.  The library links the CUDA runtime
-statically and reaches the driver's tensor-map encoder through the runtime's
+statically and reaches the CUDA driver's tensor-map encoder through the runtime's
 driver entry-point query, so it loads on a machine without a GPU.
 """
 from __future__ import annotations
