@@ -120,6 +120,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *     FA_ERR_DEVICE_TIMEOUT and clears it.  fa_check_device_status reads
  *     fa_fwd's own status word, not this one.
  *   - fp32 inputs run the fp32 kernel, which needs no scratch.
+ *   - bf16 problems whose 128-row tiles all fit on the GPU at once
+ *     (B * H * ceil(N / 128) <= SM count) run the one-tile kernel, the rest
+ *     the two-tile kernel (fa_fwd's schedule-based choice keeps a host-side
+ *     cache, which this entry point does not).
  */
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                    int64_t B, int64_t H, int64_t N, int64_t d,

@@ -30,9 +30,8 @@ int fa_test_skip_one_arrival(void);
  * fa_fwd_host launch from now on in this process: 0 (the default) the one
  * fa_fwd_kernel_choice names for the shape, 1 always the two-tile kernel,
  * 2 always the one-tile kernel.  Both compute the same result; the
- * hook lets tests check each on every shape.  fa_fwd_noalloc always uses the
- * two-tile kernel.  Returns FA_OK, or FA_ERR_INVALID_ARGUMENT for any other
- * value.
+ * hook lets tests check each on every shape; it applies to fa_fwd_noalloc
+ * too.  Returns FA_OK, or FA_ERR_INVALID_ARGUMENT for any other value.
  */
 int fa_test_force_forward_kernel(int which);
 

@@ -44,12 +44,14 @@ def _outputs(q):
     return o, lse
 
 
+@pytest.mark.parametrize("which", [0, 1, 2], ids=["by_size", "two_tile", "one_tile"])
 @pytest.mark.parametrize("dtype,d,N", [(torch.bfloat16, 128, 1100), (torch.bfloat16, 64, 700),
                                        (torch.float32, 64, 300)])
 @pytest.mark.parametrize("causal", [True, False])
-def test_noalloc_matches_oracle_and_fa_fwd_twice(dtype, d, N, causal):
+def test_noalloc_matches_oracle_and_fa_fwd_twice(dtype, d, N, causal, which, force_kernel):
     fa_build.build()
     lib = fa.library()
+    force_kernel(which)
     torch.cuda.set_device(0)
     qc, kc, vc = W.random_qkv(2, 4, N, d, dtype, seed=53 + d)
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
@@ -73,9 +75,11 @@ def test_noalloc_matches_oracle_and_fa_fwd_twice(dtype, d, N, causal):
         assert (lse - l_ref).abs().max().item() <= LSE_MAX_ABS
 
 
-def test_noalloc_timeout_is_reported_and_cleared():
+@pytest.mark.parametrize("which", [1, 2], ids=["two_tile", "one_tile"])
+def test_noalloc_timeout_is_reported_and_cleared(which, force_kernel):
     fa_build.build()
     lib = fa.library()
+    force_kernel(which)
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream().cuda_stream
     qc, kc, vc = W.random_qkv(1, 2, 512, 128, torch.bfloat16, seed=71)

@@ -515,6 +515,7 @@ struct NoAllocDevice {
     int sm_count = 0;
     int cc_major = 0;
     bool smem_raised[4] = {false, false, false, false};
+    bool tile_smem_raised[4] = {false, false, false, false};
 };
 NoAllocDevice g_noalloc_dev[kMaxDevices];
 
@@ -593,6 +594,46 @@ int launch_bf16_noalloc(NoAllocDevice* st, int slot, const void* q, const void* 
     return FA_OK;
 }
 
+// The one-tile kernel with the no-alloc scratch (same queue and status words).
+template <int D, bool kCausal>
+int launch_bf16_tile_noalloc(NoAllocDevice* st, int slot, const void* q, const void* k, const void* v, void* o,
+                             float* lse, int64_t bh, int64_t n, float scale, cudaStream_t stream) {
+    using L = fa::tc1::Layout<D>;
+    auto kernel = fa::tc1::fa_fwd_bf16_tile_kernel<D, kCausal>;
+    if (!st->tile_smem_raised[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+        std::lock_guard<std::mutex> lock(g_mu);
+        st->tile_smem_raised[slot] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = encode_tile_map(&tq, q, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tk, k, bh, n, D)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tv, v, bh, n, D)) != FA_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(st->scratch + kNoAllocQueueWord, 0, kNoAllocQueueWords * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc queue words)");
+
+    fa::tc::Params p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.status = reinterpret_cast<int*>(st->scratch + kNoAllocStatusWord);
+    p.sched = st->scratch + kNoAllocQueueWord;
+    p.bh = static_cast<int>(bh);
+    p.n = static_cast<int>(n);
+    p.num_qblocks = static_cast<int>((n + fa::tc::kBlockM - 1) / fa::tc::kBlockM);  // 128-row units
+    p.num_kblocks = static_cast<int>((n + fa::tc::kBlockN - 1) / fa::tc::kBlockN);
+    p.num_units = p.bh * p.num_qblocks;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.skip_one_arrival = g_skip_one_arrival.exchange(0);
+    p.clock = nullptr;
+    const int grid = p.num_units < st->sm_count ? p.num_units : st->sm_count;
+    kernel<<<grid, fa::tc1::kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the one-tile bf16 attention kernel (no-alloc)");
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
@@ -634,6 +675,17 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
     if (dtype == FA_DTYPE_BF16) {
         if (st->cc_major != 10)
             return fail(FA_ERR_UNSUPPORTED, "the bf16 kernel needs an sm_100 (B200-class) GPU");
+        // the one-tile kernel when every 128-row tile has its own SM (the choice
+        // fa_fwd makes by a schedule simulation keeps host state; this rule
+        // keeps none and agrees with it there)
+        const int force = g_force_forward_kernel.load();
+        const int64_t tiles = bh * ((N + fa::tc::kBlockM - 1) / fa::tc::kBlockM);
+        if (force == 2 || (force == 0 && tiles <= st->sm_count)) {
+            if (d == 128) return c ? launch_bf16_tile_noalloc<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
+                                   : launch_bf16_tile_noalloc<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
+            return c ? launch_bf16_tile_noalloc<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
+                     : launch_bf16_tile_noalloc<64, false>(st, 3, q, k, v, o, lse, bh, N, scale, s);
+        }
         if (d == 128) return c ? launch_bf16_noalloc<128, true>(st, 0, q, k, v, o, lse, bh, N, scale, s)
                                : launch_bf16_noalloc<128, false>(st, 1, q, k, v, o, lse, bh, N, scale, s);
         return c ? launch_bf16_noalloc<64, true>(st, 2, q, k, v, o, lse, bh, N, scale, s)
